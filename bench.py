@@ -1,0 +1,375 @@
+"""Benchmark: one step = the whole hot path (pooled block scores -> max-based threshold + CSR ->
+block-sparse attention) over one seeded synthetic prefill, through the C ABI.
+
+Default workload: the 131072-token Llama-3-8B-shaped layer (bf16, Hq 32 / Hkv 8, D 128,
+block 128, alpha 0.1, 0.2% vertical columns).  Inputs (Q+K+V = 1.6 GB) are larger than L2, so
+no L2 flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  `value` is the dense-equivalent throughput of the whole step:
+2 * Hq * D * sum(N^2) FLOP (causal dense attention) / step time, summed over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own copy of the workload (the
+prefill's (sequence, KV-head) units are independent; no data-path collective), timed on the
+device and reduced as the max over ranks -> weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gen import WORKLOADS, default_workers, generate  # noqa: E402
+
+METRIC = "sparse prefill-attn ms & dense-equiv TFLOP/s at 32K/128K; search ms; density"
+DEFAULT_WORKLOAD = "llama8b_bf16_n131072"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 10  # plan+pool+score, plan+count+scan+emit, plan+order+attention
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def dense_flops(w) -> float:
+    return float(sum(2.0 * w.hq * w.d * n * n for n in w.seqlens))
+
+
+def pairs(w) -> int:
+    return sum((-(-n // w.block)) * (-(-n // w.block) + 1) // 2 for n in w.seqlens)
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, max clock, throttle reasons)."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, device):
+    import dynamic_block_sparse_pooled_b200 as fpx
+
+    w = WORKLOADS[args.workload]
+    if args.alpha is not None:
+        w = w.with_(alpha=args.alpha)
+    data = generate(w, workers=default_workers())
+    cu = data["cu_seqlens"]
+    host = {k: data[k].contiguous().pin_memory() for k in ("q", "k", "v")}
+    dev = {k: host[k].to(device, non_blocking=True) for k in host}
+    for k in ("q_scale", "k_scale", "v_scale"):
+        dev[k] = data[k].to(device) if data[k] is not None else None
+    torch.cuda.synchronize(device)
+
+    stream = torch.cuda.current_stream(device)
+    pf = fpx.problem(dev["q"], dev["k"], w.block, cu, 0.0, dev["q_scale"], dev["k_scale"],
+                     dev["v_scale"])
+    ws = fpx.workspace(pf, -1, device)
+    scores = torch.empty(w.hq * pf.tri, dtype=torch.float32, device=device)
+    row_ptr = torch.empty(pf.rows + 1, dtype=torch.int32, device=device)
+    col_idx = torch.empty(max(1, w.hq * pf.tri), dtype=torch.int32, device=device)
+    nnz = torch.empty(1, dtype=torch.int64, device=device)
+    o = torch.empty(dev["q"].shape, dtype=torch.bfloat16 if w.dtype != "f32" else torch.float32,
+                    device=device)
+    lse = torch.empty((w.hq, w.total_tokens), dtype=torch.float32, device=device)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(timing=None):
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        e0.record(stream)
+        fpx.block_scores(pf, dev["q"], dev["k"], ws, scores=scores)
+        fpx.select(pf, scores, w.alpha, ws, w.sink_blocks, w.window_blocks, row_ptr=row_ptr,
+                   col_idx=col_idx, nnz=nnz)
+        e1.record(stream)
+        fpx.sparse_prefill(pf, dev["q"], dev["k"], dev["v"], row_ptr, col_idx, ws, o=o, lse=lse)
+        e2.record(stream)
+        if timing is not None:
+            timing.append((e0, e1, e2))
+
+    for _ in range(args.warmup):
+        step()
+    st = fpx.status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    n_kept = int(nnz.item())
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    timing = []
+    t_start, t_end = ev(), ev()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(timing)
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    search_ms = [a.elapsed_time(b) for a, b, c in timing]
+    attn_ms = [b.elapsed_time(c) for a, b, c in timing]
+    st = fpx.status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed steps")
+
+    # end to end through the public API: pinned host Q/K/V -> device, whole path, O + LSE -> host
+    host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    torch.cuda.synchronize(device)
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(e2e_steps):
+        for k in ("q", "k", "v"):
+            dev[k].copy_(host[k], non_blocking=True)
+        step()
+        host_o.copy_(o, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+    d2h = host_o.numel() * host_o.element_size() + host_lse.numel() * host_lse.element_size()
+
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    ms_step = total_ms / args.steps
+    flops = dense_flops(w)
+    tri = pairs(w)
+    density = n_kept / (w.hq * tri)
+    attn_avg = statistics.mean(attn_ms)
+    exec_flops = 4.0 * w.block * w.block * w.d * n_kept
+    pk, pk_kind = peaks()
+    peak_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if w.dtype == "e4m3":
+        peak_tf *= 2.0  # fp8 dense is twice bf16 (nominal ratio)
+    achieved = exec_flops / (attn_avg * 1e-3) / 1e12
+    search_bytes = (dev["q"].numel() * dev["q"].element_size() +
+                    dev["k"].numel() * dev["k"].element_size() +
+                    2 * 4 * w.hq * tri + 4 * (pf.rows + 1) + 4 * n_kept)
+    res = {
+        "metric": METRIC,
+        "value": round(world * flops / (ms_step * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s (dense-equivalent causal attention, whole step)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded generator: RoPE + sink + verticals + slash)",
+        "config": {"workload": w.name, "seqlens": list(w.seqlens), "hq": w.hq, "hkv": w.hkv,
+                   "d": w.d, "block": w.block, "alpha": w.alpha, "sink_blocks": w.sink_blocks,
+                   "window_blocks": w.window_blocks,
+                   "l2": "inputs (Q+K+V) larger than L2; no flush",
+                   "parallelism": f"replica x{world} (independent prefills)"},
+        "attn_ms": round(attn_avg, 4),
+        "search_ms": round(statistics.mean(search_ms), 4),
+        "attn_dense_equiv_tflops": round(flops / (attn_avg * 1e-3) / 1e12, 3),
+        "density": round(density, 6), "nnz": n_kept,
+        "search_gbs": round(search_bytes / (statistics.mean(search_ms) * 1e-3) / 1e9, 1),
+        "search_hbm_frac": round(search_bytes / (statistics.mean(search_ms) * 1e-3) / 1e9
+                                 / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), 4),
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(achieved, 2),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                     "peak_kind": f"{pk_kind} bf16 sustained" + (" x2 (fp8)" if w.dtype == "e4m3" else ""),
+                     "traffic": None,
+                     "per_launch": "executed FLOP = 4*B^2*D*nnz (every kept 128x128 tile)"},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3),
+                "unit": "TFLOP/s (dense-equivalent, host buffers, copies included)",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    return res, w, data
+
+
+# ---------------------------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------------------------
+
+def oracle_sample(w, data, budget_s: float = 20.0):
+    """Times the CPU oracle on a bounded sample of the workload: the pooled scores and the
+    selection of one sequence x one head, then exact attention for whole query blocks of that
+    head, last blocks first, until ~budget_s.  Returns (dense-equiv FLOP done, seconds, text)."""
+    from gen import dequantised
+    from oracle import fpx_oracle as O
+
+    s_idx = int(np.argmax(w.seqlens))
+    n = w.seqlens[s_idx]
+    a = int(data["cu_seqlens"][s_idx])
+    g = w.hq // w.hkv
+    sl = slice(a, a + n)
+    q = dequantised(data["q"][sl, :1], None if data["q_scale"] is None else data["q_scale"][:1])
+    k = dequantised(data["k"][sl, :1], None if data["k_scale"] is None else data["k_scale"][:1])
+    v = dequantised(data["v"][sl, :1], None if data["v_scale"] is None else data["v_scale"][:1])
+    cu = np.array([0, n])
+    t0 = time.perf_counter()
+    sc = O.block_scores(q, k, cu, w.block)
+    keeps, _ = O.select(sc, w.alpha, w.sink_blocks, w.window_blocks)
+    rp, ci = O.to_csr(keeps)
+    nb = keeps[0].shape[1]
+    flop = 0.0
+    done = 0
+    for I in range(nb - 1, -1, -1):
+        O.attention(q, k, v, cu, w.block, rp, ci, blocks=[(0, 0, I)])
+        flop += sum(4.0 * w.d * (I * w.block + r + 1) for r in range(min(w.block, n - I * w.block)))
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    text = (f"sequence {s_idx} (N={n}), Q head 0 (KV head 0, group {g}): pooled scores + selection"
+            f" of all {nb} query blocks, exact attention of the last {done} query blocks")
+    return flop, dt, text
+
+
+def cpu_cores() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((x.get("num_threads", 1) for x in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    w = WORKLOADS[args.workload]
+    if args.alpha is not None:
+        w = w.with_(alpha=args.alpha)
+    data = generate(w, workers=default_workers())
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, data, budget)
+    vals = []
+    text = ""
+    for _ in range(args.steps):
+        flop, dt, text = oracle_sample(w, data, budget)
+        vals.append(flop / dt / 1e12)
+    v = statistics.mean(vals)
+    unit = "TFLOP/s (dense-equivalent causal attention, whole step)"
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name},
+        "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": text},
+        "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--alpha", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    res, w, data = run_ours(args, rank, world, device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flop, dt, text = oracle_sample(w, data, 20.0)
+        res["cpu_baseline"] = {"value": flop / dt / 1e12,
+                               "unit": "TFLOP/s (dense-equivalent causal attention)",
+                               "cores": cpu_cores(), "kind": "oracle", "sample": text,
+                               "seconds": round(dt, 2)}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+// fpx_api.cu -- the C ABI declared in include/fpx.h: host-side validation, workspace layout and
+// the launch sequence of every stage.  Nothing here allocates, frees or synchronises (except
+// fpx_query_status, which synchronises the stream it is given).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "fpx_internal.h"
+
+using namespace fpx;
+
+namespace {
+
+struct Sizes {
+  int64_t nb = 0;   // NB
+  int64_t tri = 0;  // TRI
+};
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validates the problem description; fills sizes.  Everything here runs on the host.
+fpx_status check_problem(const fpx_problem* p, Sizes* sz) {
+  if (!p) return FPX_ERR_INVALID_ARG;
+  if (p->dtype != FPX_F32 && p->dtype != FPX_BF16 && p->dtype != FPX_E4M3)
+    return FPX_ERR_UNSUPPORTED;
+  if (p->d != 64 && p->d != 128) return FPX_ERR_UNSUPPORTED;
+  if (!is_pow2(p->block) || p->block < 16 || p->block > 128) return FPX_ERR_UNSUPPORTED;
+  if (p->hq < 1 || p->hkv < 1 || p->hq % p->hkv != 0) return FPX_ERR_INVALID_ARG;
+  if (p->total_tokens < 0 || p->num_seqs < 1) return FPX_ERR_INVALID_ARG;
+  if ((p->cu_seqlens_d == nullptr) != (p->cu_seqlens_h == nullptr)) return FPX_ERR_INVALID_ARG;
+  if (p->dtype == FPX_E4M3 && (!p->q_scale_d || !p->k_scale_d || !p->v_scale_d))
+    return FPX_ERR_INVALID_ARG;
+  if (std::isnan(p->softmax_scale) || std::isinf(p->softmax_scale)) return FPX_ERR_INVALID_ARG;
+  Sizes s;
+  if (!p->cu_seqlens_h) {
+    if (p->num_seqs != 1) return FPX_ERR_INVALID_ARG;
+    s.nb = (static_cast<int64_t>(p->total_tokens) + p->block - 1) / p->block;
+    s.tri = s.nb * (s.nb + 1) / 2;
+  } else {
+    const int32_t* cu = p->cu_seqlens_h;
+    if (cu[0] != 0 || cu[p->num_seqs] != p->total_tokens) return FPX_ERR_INVALID_ARG;
+    for (int i = 0; i < p->num_seqs; ++i) {
+      const int64_t n = static_cast<int64_t>(cu[i + 1]) - cu[i];
+      if (n < 0) return FPX_ERR_INVALID_ARG;
+      const int64_t nb = (n + p->block - 1) / p->block;
+      s.nb += nb;
+      s.tri += nb * (nb + 1) / 2;
+    }
+  }
+  // int32 CSR (row_ptr, col_idx) and int32 grid / row indices
+  if (s.nb * p->hq >= INT32_MAX || s.tri * p->hq >= INT32_MAX) return FPX_ERR_UNSUPPORTED;
+  *sz = s;
+  return FPX_OK;
+}
+
+ProblemDesc make_desc(const fpx_problem* p, const Sizes& s) {
+  ProblemDesc d;
+  d.cu = p->cu_seqlens_d;
+  d.num_seqs = p->num_seqs;
+  d.total_tokens = p->total_tokens;
+  d.hq = p->hq;
+  d.hkv = p->hkv;
+  d.group = p->hq / p->hkv;
+  d.d = p->d;
+  d.block = p->block;
+  d.nb_total = static_cast<int32_t>(s.nb);
+  d.tri_total = s.tri;
+  d.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(p->d));
+  const bool fp8 = p->dtype == FPX_E4M3;
+  d.q_scale = fp8 ? p->q_scale_d : nullptr;
+  d.k_scale = fp8 ? p->k_scale_d : nullptr;
+  d.v_scale = fp8 ? p->v_scale_d : nullptr;
+  return d;
+}
+
+size_t scratch_bytes(const fpx_problem* p, const Sizes& s, int which) {
+  const size_t R = static_cast<size_t>(s.nb) * p->hq;
+  switch (which) {
+    case 0:  // pooled Q and K, fp32
+      return align_up(sizeof(float) * s.nb * p->hq * p->d, 256) +
+             align_up(sizeof(float) * s.nb * p->hkv * p->d, 256);
+    case 1:  // row max, keep counts, overflow flag
+      return align_up(sizeof(float) * R, 256) + align_up(sizeof(int32_t) * R, 256) + 256;
+    case 2:  // tile schedule
+      return align_up(sizeof(int32_t) * R, 256);
+    default:
+      return 0;
+  }
+}
+
+size_t ws_bytes_for(const fpx_problem* p, const Sizes& s, int which) {
+  return scratch_offset(p->num_seqs) + scratch_bytes(p, s, which);
+}
+
+fpx_status check_ws(const fpx_problem* p, const Sizes& s, int which, void* ws, size_t ws_bytes) {
+  if (!ws) return FPX_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return FPX_ERR_ALIGNMENT;
+  if (ws_bytes < ws_bytes_for(p, s, which)) return FPX_ERR_CAPACITY;
+  return FPX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fpx_num_blocks(const fpx_problem* p) {
+  Sizes s;
+  return check_problem(p, &s) == FPX_OK ? static_cast<size_t>(s.nb) : 0;
+}
+size_t fpx_scores_elems(const fpx_problem* p) {
+  Sizes s;
+  return check_problem(p, &s) == FPX_OK ? static_cast<size_t>(s.tri) * p->hq : 0;
+}
+size_t fpx_rows(const fpx_problem* p) {
+  Sizes s;
+  return check_problem(p, &s) == FPX_OK ? static_cast<size_t>(s.nb) * p->hq : 0;
+}
+size_t fpx_max_nnz(const fpx_problem* p) { return fpx_scores_elems(p); }
+
+size_t fpx_workspace_bytes(const fpx_problem* p, int which) {
+  Sizes s;
+  if (check_problem(p, &s) != FPX_OK) return 0;
+  if (which >= 0 && which <= 2) return ws_bytes_for(p, s, which);
+  if (which != -1) return 0;
+  size_t m = 0;
+  for (int w = 0; w <= 2; ++w) m = ws_bytes_for(p, s, w) > m ? ws_bytes_for(p, s, w) : m;
+  return m;
+}
+
+fpx_status fpx_clear_status(void* ws, fpx_stream_t stream) {
+  if (!ws) return FPX_ERR_INVALID_ARG;
+  return cudaMemsetAsync(ws, 0, kStatusBytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FPX_OK
+             : FPX_ERR_CUDA;
+}
+
+fpx_status fpx_query_status(const void* ws, fpx_stream_t stream) {
+  if (!ws) return FPX_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FPX_ERR_CUDA;
+  StatusBlock h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return FPX_ERR_CUDA;
+  return static_cast<fpx_status>(h.code);
+}
+
+const char* fpx_status_string(fpx_status s) {
+  switch (s) {
+    case FPX_OK: return "ok";
+    case FPX_ERR_INVALID_ARG: return "invalid argument";
+    case FPX_ERR_UNSUPPORTED: return "unsupported dtype, head dim, block size or size";
+    case FPX_ERR_ALIGNMENT: return "misaligned pointer";
+    case FPX_ERR_CAPACITY: return "capacity too small";
+    case FPX_ERR_CUDA: return "CUDA error";
+    case FPX_ERR_TIMEOUT: return "device-side wait timed out";
+    case FPX_ERR_DEVICE_INPUT: return "malformed device input (cu_seqlens or CSR)";
+  }
+  return "unknown status";
+}
+
+int fpx_attention_path(const fpx_problem* p) {
+  Sizes s;
+  if (check_problem(p, &s) != FPX_OK) return -1;
+  return attn_tc_supported(make_desc(p, s), p->dtype) ? 1 : 0;
+}
+
+fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, float* scores,
+                            void* ws, size_t ws_bytes, fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if ((rc = check_ws(p, sz, 0, ws, ws_bytes)) != FPX_OK) return rc;
+  if (p->total_tokens > 0 && (!q || !k || !scores)) return FPX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(scores, 4)) return FPX_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const ProblemDesc d = make_desc(p, sz);
+  StatusBlock* st = static_cast<StatusBlock*>(ws);
+  const SeqTables t = seq_tables_at(ws, p->num_seqs);
+  char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
+  float* qbar = reinterpret_cast<float*>(scratch);
+  float* kbar = reinterpret_cast<float*>(scratch + align_up(sizeof(float) * sz.nb * p->hq * p->d, 256));
+  if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (sz.nb == 0) return FPX_OK;
+  if (launch_pool(d, p->dtype, q, k, qbar, kbar, t, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (launch_score(d, p->dtype, qbar, kbar, scores, t, s) != cudaSuccess) return FPX_ERR_CUDA;
+  return FPX_OK;
+}
+
+fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, int32_t sink_blocks,
+                      int32_t window_blocks, int32_t* row_ptr, int32_t* col_idx,
+                      int64_t col_capacity, int64_t* nnz_d, void* ws, size_t ws_bytes,
+                      fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if ((rc = check_ws(p, sz, 1, ws, ws_bytes)) != FPX_OK) return rc;
+  if (std::isnan(alpha) || alpha < 0.f) return FPX_ERR_INVALID_ARG;
+  if (sink_blocks < 0 || window_blocks < 0 || col_capacity < 0) return FPX_ERR_INVALID_ARG;
+  if (!row_ptr) return FPX_ERR_INVALID_ARG;
+  if (sz.tri > 0 && (!scores || (!col_idx && col_capacity > 0))) return FPX_ERR_INVALID_ARG;
+  if (!aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(nnz_d, 8))
+    return FPX_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const ProblemDesc d = make_desc(p, sz);
+  StatusBlock* st = static_cast<StatusBlock*>(ws);
+  const SeqTables t = seq_tables_at(ws, p->num_seqs);
+  const size_t R = static_cast<size_t>(sz.nb) * p->hq;
+  char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
+  float* rowmax = reinterpret_cast<float*>(scratch);
+  int32_t* counts = reinterpret_cast<int32_t*>(scratch + align_up(sizeof(float) * R, 256));
+  int* overflow = reinterpret_cast<int*>(scratch + align_up(sizeof(float) * R, 256) +
+                                         align_up(sizeof(int32_t) * R, 256));
+  if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
+  // window / sink beyond any row are equivalent to "all": clamp so the device compare stays
+  // in range
+  const int sink = sink_blocks > d.nb_total ? d.nb_total + 1 : sink_blocks;
+  const int window = window_blocks > d.nb_total ? d.nb_total + 1 : window_blocks;
+  if (launch_select(d, scores, alpha, sink, window, row_ptr, col_idx, col_capacity, nnz_d, rowmax,
+                    counts, overflow, t, st, s) != cudaSuccess)
+    return FPX_ERR_CUDA;
+  return FPX_OK;
+}
+
+fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k, const void* v,
+                              const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                              float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if ((rc = check_ws(p, sz, 2, ws, ws_bytes)) != FPX_OK) return rc;
+  if (p->total_tokens > 0 && (!q || !k || !v || !o || !row_ptr)) return FPX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
+    return FPX_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const ProblemDesc d = make_desc(p, sz);
+  StatusBlock* st = static_cast<StatusBlock*>(ws);
+  const SeqTables t = seq_tables_at(ws, p->num_seqs);
+  char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
+  int32_t* order = reinterpret_cast<int32_t*>(scratch);
+  if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (sz.nb == 0) return FPX_OK;
+  if (launch_order(d, t, order, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (attn_tc_supported(d, p->dtype)) {
+    bool encode_failed = false;
+    cudaError_t e = launch_attn_tc(d, p->dtype, q, k, v, row_ptr, col_idx, o, lse, t, order, st, s,
+                                   &encode_failed);
+    if (encode_failed) return FPX_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? FPX_OK : FPX_ERR_CUDA;
+  }
+  return launch_attn_simt(d, p->dtype, q, k, v, row_ptr, col_idx, o, lse, t, order, st, s) == cudaSuccess
+             ? FPX_OK
+             : FPX_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,38 @@
+// fpx_internal.h -- host-side declarations shared by the fpx translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "fpx_common.cuh"
+
+namespace fpx {
+
+// Stage 0 building block, shared by all entry points: per-sequence tables + cu_seqlens checks.
+cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cudaStream_t s);
+
+// fpx_block_scores: pool Q and K (fp32 means into qbar / kbar), then score pooled pairs.
+cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
+                        float* qbar, float* kbar, SeqTables t, cudaStream_t s);
+cudaError_t launch_score(const ProblemDesc& p, fpx_dtype dt, const float* qbar, const float* kbar,
+                         float* scores, SeqTables t, cudaStream_t s);
+
+// fpx_select: row max + keep count, scan into row_ptr, emit col_idx.
+cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
+                          int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
+                          int64_t* nnz_d, float* rowmax, int32_t* counts, int* overflow,
+                          SeqTables t, StatusBlock* st, cudaStream_t s);
+
+// fpx_sparse_prefill: tile schedule, then one of the two attention kernels.
+cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, cudaStream_t s);
+cudaError_t launch_attn_simt(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
+                             const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                             void* o, float* lse, SeqTables t, const int32_t* order,
+                             StatusBlock* st, cudaStream_t s);
+bool attn_tc_supported(const ProblemDesc& p, fpx_dtype dt);
+// Returns cudaSuccess or the first error; `encode_failed` is set if a tensor map was rejected.
+cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
+                           const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                           void* o, float* lse, SeqTables t, const int32_t* order,
+                           StatusBlock* st, cudaStream_t s, bool* encode_failed);
+
+}  // namespace fpx

@@ -1,0 +1,162 @@
+/*
+ * fpx.h -- C ABI of the dynamic block-sparse pooled prefill attention library (sm_100a).
+ *
+ * The library runs, for one causal prefill (optionally a packed varlen batch), the three stages
+ * of FlashPrefill ("FlashPrefill: Instantaneous Pattern Discovery and Thresholding for
+ * Ultra-Fast Long-Context Prefilling", App. B "Detailed Implementation"):
+ *
+ *   fpx_block_scores   Instantaneous Pattern Discovery: mean-pool Q and K over B-token blocks
+ *                      and score every pooled query block against every causally valid pooled
+ *                      key block (§3 Method, "Block Approximation for Kernel Optimization").
+ *   fpx_select         Max-based Dynamic Thresholding and Block Selection: keep block J of row I
+ *                      iff its row-normalised score reaches alpha times the row maximum, OR the
+ *                      sink / local-window masks, restricted to J <= I; compress to CSR (§3,
+ *                      "Max-based Dynamic Thresholding"; App. B).
+ *   fpx_sparse_prefill Block Sparse Attention: exact online-softmax attention over the kept
+ *                      blocks only, token-causal inside the diagonal block; O and per-row LSE
+ *                      (App. B, "Block Sparse Attention").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layouts.  Q is [T, Hq, D], K and V are [T, Hkv, D], row-major and contiguous ("packed THD"),
+ *   base addresses 16-byte aligned (fp8 / bf16 / fp32 elements).  Query head h reads KV head
+ *   h / (Hq / Hkv).  A packed batch is described by cu_seqlens (cu[0] = 0, non-decreasing,
+ *   cu[S] = T); blocks restart at every sequence start and never cross a sequence boundary.
+ *   nb_s = ceil(n_s / B) blocks per sequence, NB = sum_s nb_s, TRI = sum_s nb_s (nb_s + 1) / 2.
+ * Scores.  fp32, triangular-packed, one row per (h, s, I): row (h, s, I) starts at element
+ *   h * TRI + tri_base[s] + I (I + 1) / 2 and holds J = 0..I, where tri_base[s] is the sum of
+ *   nb (nb + 1) / 2 over the sequences before s.
+ * CSR.  Rows r = h * NB + block_base[s] + I (i.e. ordered (h, s, I)); row_ptr int32 [R + 1]
+ *   with R = Hq * NB; col_idx int32 lists key-block indices local to the sequence, ascending.
+ * Ownership.  The caller owns every buffer.  No entry point allocates, frees or synchronises
+ *   (except fpx_query_status, which synchronises the stream it is given).  All work is enqueued
+ *   on the caller's stream; the library keeps no state between calls and is re-entrant.
+ * Workspaces.  Each entry point takes a device workspace of at least fpx_workspace_bytes()
+ *   bytes (256-byte aligned).  Its first 256 bytes are a status block: kernels record the first
+ *   device-side error there (bounded-wait timeout, malformed cu_seqlens or CSR, capacity); the
+ *   record is sticky until fpx_clear_status().  One buffer of the largest size may serve all
+ *   three stages on one stream.  Zero it (fpx_clear_status) before first use.
+ * Errors.  Argument errors are found on the host before anything is launched and return a
+ *   negative fpx_status; launch failures return FPX_ERR_CUDA.  Device-side conditions are read
+ *   with fpx_query_status().  Nothing traps on the device and no exception crosses the ABI.
+ */
+#ifndef FPX_H_
+#define FPX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st* fpx_stream_t;
+
+typedef enum {
+  FPX_OK = 0,
+  FPX_ERR_INVALID_ARG = -1,  /* null pointer, bad shape, bad cu_seqlens, NaN/negative alpha  */
+  FPX_ERR_UNSUPPORTED = -2,  /* dtype / head dim / block size / index range not supported    */
+  FPX_ERR_ALIGNMENT = -3,    /* a pointer is not aligned as documented                      */
+  FPX_ERR_CAPACITY = -4,     /* workspace or col_idx capacity too small                      */
+  FPX_ERR_CUDA = -5,         /* a CUDA runtime / driver call or a launch failed              */
+  FPX_ERR_TIMEOUT = -6,      /* a bounded device-side wait expired (recorded in the status)  */
+  FPX_ERR_DEVICE_INPUT = -7  /* device data was malformed (cu_seqlens, CSR index > row block) */
+} fpx_status;
+
+typedef enum { FPX_F32 = 0, FPX_BF16 = 1, FPX_E4M3 = 2 } fpx_dtype;
+
+typedef struct {
+  int32_t num_seqs;            /* >= 1 (1 when cu_seqlens_d is NULL)                           */
+  const int32_t* cu_seqlens_d; /* device [num_seqs + 1]; NULL => one sequence of total_tokens   */
+  const int32_t* cu_seqlens_h; /* host mirror of cu_seqlens_d (sizes grids and outputs); NULL
+                                  iff cu_seqlens_d is NULL.  Must equal the device copy.        */
+  int32_t total_tokens;        /* T >= 0                                                        */
+  int32_t hq, hkv;             /* query / KV heads, hq % hkv == 0, both >= 1                    */
+  int32_t d;                   /* head dim: 64 or 128                                           */
+  int32_t block;               /* B: power of two in [16, 128]                                  */
+  fpx_dtype dtype;             /* storage type of Q, K, V                                       */
+  const float* q_scale_d;      /* FPX_E4M3 only: device fp32 [hq] dequantisation scales, else NULL */
+  const float* k_scale_d;      /* FPX_E4M3 only: device fp32 [hkv]                              */
+  const float* v_scale_d;      /* FPX_E4M3 only: device fp32 [hkv]                              */
+  float softmax_scale;         /* scale of the dequantised dot products; <= 0 => 1/sqrt(d)      */
+} fpx_problem;
+
+/* Sizes.  Each returns 0 for an invalid problem. */
+size_t fpx_num_blocks(const fpx_problem* p);   /* NB                                           */
+size_t fpx_scores_elems(const fpx_problem* p); /* hq * TRI fp32 elements of the scores buffer  */
+size_t fpx_rows(const fpx_problem* p);         /* R = hq * NB; row_ptr has R + 1 entries       */
+size_t fpx_max_nnz(const fpx_problem* p);      /* hq * TRI: col_idx entries when alpha == 0    */
+
+/* Workspace bytes for stage `which`: 0 = fpx_block_scores, 1 = fpx_select,
+ * 2 = fpx_sparse_prefill, -1 = the maximum of the three. */
+size_t fpx_workspace_bytes(const fpx_problem* p, int which);
+
+/* Zero the status block of a workspace (async on `stream`). */
+fpx_status fpx_clear_status(void* ws, fpx_stream_t stream);
+
+/* Synchronise `stream`, then return the first device-side error recorded in the workspace's
+ * status block (FPX_OK if none).  The record is left in place. */
+fpx_status fpx_query_status(const void* ws, fpx_stream_t stream);
+
+const char* fpx_status_string(fpx_status s);
+
+/*
+ * Stage 1 -- Instantaneous Pattern Discovery (FlashPrefill §3 "Instantaneous Pattern Discovery"
+ * and "Block Approximation for Kernel Optimization"; App. B).
+ *   q, k    device, [T, Hq, D] and [T, Hkv, D] in p->dtype (e4m3 codes for FPX_E4M3).
+ *   scores  device fp32 [hq * TRI] (layout above):
+ *           scores(h, s, I, J) = scale * <mean_{i in I} q_i, mean_{j in J} k_j>  for J <= I,
+ *           means over the valid rows of each block (a tail block averages the rows it has),
+ *           scale = softmax_scale (dequantised: times q_scale[h] * k_scale[h / g] for e4m3).
+ *   ws      device workspace >= fpx_workspace_bytes(p, 0); holds the pooled vectors.
+ */
+fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, float* scores,
+                            void* ws, size_t ws_bytes, fpx_stream_t stream);
+
+/*
+ * Stage 2 -- Max-based Dynamic Thresholding and Block Selection (FlashPrefill §3 "Max-based
+ * Dynamic Thresholding"; App. B "Dynamic Thresholding and Block Selection").
+ *   For each row (h, s, I) with m = max_{J <= I} scores(h, s, I, J), key block J <= I is kept iff
+ *     alpha == 0  or  expf(score - m) >= alpha  (the row-softmax ratio P_IJ / max_J P_IJ)
+ *     or J < sink_blocks  or  J > I - window_blocks.
+ *   alpha >= 0 (NaN rejected); sink_blocks, window_blocks >= 0.
+ *   row_ptr   device int32 [R + 1], written (row_ptr[0] = 0, row_ptr[R] = nnz).
+ *   col_idx   device int32 [col_capacity]; kept J per row, ascending.  If nnz > col_capacity
+ *             nothing is written to col_idx and FPX_ERR_CAPACITY is recorded in the status.
+ *   nnz_d     device int64 [1] (may be NULL): total kept blocks.
+ *   ws        device workspace >= fpx_workspace_bytes(p, 1).
+ */
+fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha,
+                      int32_t sink_blocks, int32_t window_blocks, int32_t* row_ptr,
+                      int32_t* col_idx, int64_t col_capacity, int64_t* nnz_d, void* ws,
+                      size_t ws_bytes, fpx_stream_t stream);
+
+/*
+ * Stage 3 -- Block Sparse Attention (FlashPrefill App. B "Block Sparse Attention").
+ *   For Q head h and query token i (local position, block I = i / B) of sequence s:
+ *     l_j = scale * <q_i, k_j>  over key tokens j of the blocks listed in CSR row (h, s, I), j <= i
+ *     lse_i = ln sum_j exp(l_j),   o_i = sum_j exp(l_j - lse_i) v_j
+ *   (dequantised values for e4m3).  A row with no key gets o = 0 and lse = -inf.
+ *   q, k, v   device, layouts above.
+ *   row_ptr, col_idx  CSR as written by fpx_select (any CSR with indices in [0, I] and no
+ *             duplicates is accepted; an index outside [0, I] is skipped and recorded as
+ *             FPX_ERR_DEVICE_INPUT).
+ *   o         device [T, Hq, D]: bf16 for FPX_BF16 and FPX_E4M3 inputs, fp32 for FPX_F32.
+ *   lse       device fp32 [Hq, T], natural log (may be NULL).
+ *   ws        device workspace >= fpx_workspace_bytes(p, 2) (holds the tile schedule).
+ */
+fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k, const void* v,
+                              const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                              float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream);
+
+/* Which attention kernel fpx_sparse_prefill uses for this problem: 1 = the tcgen05/TMEM
+ * tensor-core mainloop (bf16 / e4m3, B = 128, D = 128), 0 = the CUDA-core kernel (fp32 and the
+ * remaining shapes). */
+int fpx_attention_path(const fpx_problem* p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FPX_H_ */

@@ -212,14 +212,16 @@ def _row_index(layouts, hq, h, s, I) -> int:
 
 def attention(q, k, v, cu_seqlens, block: int, row_ptr, col_idx,
               scale: Optional[float] = None,
-              rows: Optional[Iterable[Tuple[int, int]]] = None):
+              rows: Optional[Iterable[Tuple[int, int]]] = None,
+              blocks: Optional[Iterable[Tuple[int, int, int]]] = None):
     """Exact softmax attention over the kept blocks (FlashPrefill App. B, Block Sparse
     Attention), token causal mask applied (key position <= query position, both local to the
     sequence).  For query token t of sequence s in block I, Q head h:
         l_j = scale * <q_t, k_j>  for j in the kept blocks of row (h, s, I), j <= t
         lse_t = log sum_j exp(l_j);  o_t = sum_j exp(l_j - lse_t) v_j.
-    Returns (O [T, Hq, D], LSE [Hq, T]) in fp64 for every token, or, when ``rows`` lists
-    (h, t) pairs, (O [n, D], LSE [n]) for those pairs only."""
+    Returns (O [T, Hq, D], LSE [Hq, T]) in fp64 for every token; when ``rows`` lists (h, t)
+    pairs, (O [n, D], LSE [n]) for those pairs only; when ``blocks`` lists (h, s, I) query
+    blocks, a list of (O [rows, D], LSE [rows]) for the valid rows of each block."""
     hq, hkv, d = q.shape[1], k.shape[1], q.shape[2]
     g = hq // hkv
     sc = default_scale(d) if scale is None or scale <= 0 else float(scale)
@@ -254,6 +256,13 @@ def attention(q, k, v, cu_seqlens, block: int, row_ptr, col_idx,
         lse[empty] = -np.inf
         o[empty] = 0.0
         return o, lse
+
+    if blocks is not None:
+        out = []
+        for h, s, I in blocks:
+            nrow = min(block, layouts[s]["n"] - I * block)
+            out.append(one_block(s, h, I, np.arange(nrow)))
+        return out
 
     if rows is None:
         t_total = int(cu_seqlens[-1])

@@ -264,3 +264,20 @@ ALL_CHECKS = [
     check_attention_given_mask,
     check_varlen_equals_separate,
 ]
+
+
+def check_block_evaluation_matches_full(O):
+    seqlens = [90, 200]
+    q, k, v, cu = rand_problem(seqlens, 2, 1, 8, seed=11, scale_q=3.0)
+    res = O.prefill(q, k, v, cu, 32, 0.3)
+    picks = [(0, 0, 2), (1, 1, 6), (1, 0, 0)]
+    out = O.attention(q, k, v, cu, 32, res["row_ptr"], res["col_idx"], blocks=picks)
+    lay = O.seq_layout(cu, 32)
+    for (h, s, I), (o, lse) in zip(picks, out):
+        t0 = lay[s]["start"] + I * 32
+        n = o.shape[0]
+        assert np.abs(o - res["o"][t0:t0 + n, h]).max() < 1e-12
+        assert np.abs(lse - res["lse"][h, t0:t0 + n]).max() < 1e-12
+
+
+ALL_CHECKS.append(check_block_evaluation_matches_full)
