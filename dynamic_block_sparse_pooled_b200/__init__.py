@@ -29,7 +29,8 @@ STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "misaligned po
 # every symbol include/fpx.h declares
 EXPORTS = ("fpx_num_blocks", "fpx_scores_elems", "fpx_rows", "fpx_max_nnz", "fpx_workspace_bytes",
            "fpx_clear_status", "fpx_query_status", "fpx_status_string", "fpx_block_scores",
-           "fpx_select", "fpx_sparse_prefill", "fpx_attention_path")
+           "fpx_select", "fpx_sparse_prefill", "fpx_attention_path", "fpx_select_noalloc",
+           "fpx_select_noalloc_max_bytes")
 
 
 class FpxError(RuntimeError):
@@ -82,6 +83,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fpx_select.restype = ctypes.c_int
     lib.fpx_sparse_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.fpx_sparse_prefill.restype = ctypes.c_int
+    lib.fpx_select_noalloc.argtypes = [P, vp, f32, i32, i32, vp, vp, i64, vp, vp]
+    lib.fpx_select_noalloc.restype = ctypes.c_int
+    lib.fpx_select_noalloc_max_bytes.argtypes = []
+    lib.fpx_select_noalloc_max_bytes.restype = sz
     _lib = lib
     return lib
 
@@ -195,6 +200,26 @@ def select(pf: Prefill, scores: torch.Tensor, alpha: float, ws: torch.Tensor,
     check(load().fpx_select(pf.ptr, _ptr(scores), float(alpha), sink_blocks, window_blocks,
                             _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz), _ptr(ws), ws.numel(),
                             _stream(stream)), "fpx_select")
+    return row_ptr, col_idx, nnz
+
+
+def select_noalloc(pf: Prefill, scores: torch.Tensor, alpha: float, sink_blocks: int = 1,
+                   window_blocks: int = 1, row_ptr=None, col_idx=None, nnz=None,
+                   capacity: Optional[int] = None, stream=None):
+    """fpx_select_noalloc: fpx_select for callers that cannot provide a workspace (the scratch
+    is a fixed device array inside the library; concurrent calls on one device race on it)."""
+    dev = scores.device
+    if row_ptr is None:
+        row_ptr = torch.empty(pf.rows + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        cap = pf.struct.hq * pf.tri if capacity is None else capacity
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    cap = col_idx.numel() if capacity is None else capacity
+    if nnz is None:
+        nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    check(load().fpx_select_noalloc(pf.ptr, _ptr(scores), float(alpha), sink_blocks,
+                                    window_blocks, _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz),
+                                    _stream(stream)), "fpx_select_noalloc")
     return row_ptr, col_idx, nnz
 
 

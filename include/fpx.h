@@ -150,6 +150,31 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
                               const int32_t* row_ptr, const int32_t* col_idx, void* o,
                               float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream);
 
+/*
+ * Allocation-free variant of fpx_select (the paper has no counterpart; it exists for callers).
+ *   Some callers cannot allocate device memory where they run: a plugin whose host framework
+ *   owns all device memory and offers no scratch buffer, or latency-critical code that must not
+ *   call cudaMalloc because an allocation can synchronise the device.  This entry point takes no
+ *   workspace: the stage's scratch lives in one fixed device array inside the library of
+ *   fpx_select_noalloc_max_bytes() bytes (2 MiB), which every GPU that loads the library holds
+ *   until the process exits.  The caller still owns scores, row_ptr, col_idx and nnz_d.
+ *   Same arguments and results as fpx_select, without ws / ws_bytes.
+ *   Limits: the problem's fpx_workspace_bytes(p, 1) must not exceed the array (about 260,000
+ *   query-block rows Hq * NB for a few sequences); larger problems return FPX_ERR_CAPACITY
+ *   before anything is launched.  An invalid or unsupported problem returns FPX_ERR_INVALID_ARG.
+ *   Device-side conditions are visible through the outputs: nnz > col_capacity means nothing was
+ *   written to col_idx; device cu_seqlens that disagree with the host mirror give an empty CSR.
+ *   The first call on a device looks up the array's device address (once per device, with that
+ *   device current); make that first call before any stream capture.  All calls on a device
+ *   share the array and each call re-zeroes the part that must start at zero: calls whose work
+ *   overlaps on the GPU (unordered streams) race on it.
+ */
+fpx_status fpx_select_noalloc(const fpx_problem* p, const float* scores, float alpha,
+                              int32_t sink_blocks, int32_t window_blocks, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int64_t* nnz_d,
+                              fpx_stream_t stream);
+size_t fpx_select_noalloc_max_bytes(void);
+
 /* Which attention kernel fpx_sparse_prefill uses for this problem: 1 = the tcgen05/TMEM
  * tensor-core mainloop (bf16 / e4m3, B = 128, D = 128), 0 = the CUDA-core kernel (fp32 and the
  * remaining shapes). */
