@@ -242,8 +242,9 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
   int32_t* order = reinterpret_cast<int32_t*>(scratch);
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   if (sz.nb == 0) return FPX_OK;
-  if (launch_order(d, t, order, s) != cudaSuccess) return FPX_ERR_CUDA;
-  if (attn_tc_supported(d, p->dtype)) {
+  const bool tc = attn_tc_supported(d, p->dtype);
+  if (launch_order(d, t, order, tc, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (tc) {
     bool encode_failed = false;
     cudaError_t e = launch_attn_tc(d, p->dtype, q, k, v, row_ptr, col_idx, o, lse, t, order, st, s,
                                    &encode_failed);

@@ -1,23 +1,41 @@
 // fpx_attn_sm100.cu -- block-sparse prefill attention on the 5th-generation tensor cores
-// (FlashPrefill App. B, "Block Sparse Attention": iterate only over the selected blocks,
-// causal masking where required, online softmax with a final normalisation).
+// (FlashPrefill App. B, "Block Sparse Attention": iterate only over the selected blocks, causal
+// masking where required, online softmax with a final normalisation).
 //
-// Tile = one CSR row (Q head h, sequence s, query block I): 128 query rows x D = 128.
-//   * TMA loads the Q tile once and, for every kept key block J of the row, the K_J and V_J
-//     tiles (coordinates gathered from col_idx) into a two-stage shared-memory ring.
-//   * S = Q K_J^T runs as tcgen05.mma (M = 128, N = 128) with the fp32 accumulator in TMEM.
-//   * Each of the 128 threads owns one query row (= one TMEM lane): it reads its S row with
-//     tcgen05.ld, applies the token causal mask (diagonal block only), updates the running max
-//     and sum in the exp2 domain, rescales its O row in TMEM when the max moved, and writes P
-//     (bf16, or e4m3 for fp8 inputs) back into TMEM over S.
-//   * O += P V_J runs as tcgen05.mma with A = P read from TMEM and B = V from shared memory.
-//   * The epilogue divides O by the row sum and writes O (bf16) and the natural-log LSE.
-// Every wait is bounded (FPX_ERR_TIMEOUT is recorded and the CTA exits cleanly).
+// Work unit = two query tiles that share one KV head ("GQA head packing"): Q heads h0 = 2p and
+// h1 = 2p + 1 of KV group g, both at query block I of sequence s (128 rows x D = 128 each).
+// The CTA walks the union of the two heads' CSR rows; a key block is loaded once (TMA, gathered
+// by block index) and multiplied only by the tile(s) that kept it.
+//
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3  softmax for tile 0: one query row (= one TMEM lane) per thread
+//   warps 4-7  softmax for tile 1
+//   warp  8    tcgen05.mma issue (one thread), TMEM allocation
+//   warp  9    TMA loads (one thread): Q0/Q1 once, then K_J and V_J into 2-slot rings
+//   warps 10-11 idle (they complete the third warpgroup)
+// setmaxnreg moves registers from the third warpgroup to the two softmax warpgroups, which
+// hold a whole 128-column S row in registers.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_t (bf16 / e4m3)
+// is written over the first columns of S_t and read from TMEM by the P*V MMA.
+//
+// Per kept block the MMA thread issues S_t = Q_t K_J^T, and later O_t += P_t V_J as soon as
+// softmax t has published P_t.  It never waits on one operation while another is ready (it
+// polls K arrivals and both tiles' P barriers), so a tile that skips blocks never stalls the
+// other one and every ring slot is released as soon as its last reader is issued.  S_t for
+// the next block is issued only after O_t += P_t V for the previous one (P aliases S), so when
+// softmax t sees S_t complete, the previous P*V into O_t has completed too and O_t may be
+// rescaled in place.
+//
+// Softmax: exp2 domain, lazy rescale (the reference max only moves when the block max exceeds it
+// by more than 2^8), two passes over S in TMEM (row max, then P) so that only 32 columns are live
+// in registers at a time.  Every wait is bounded: a broken pipeline records FPX_ERR_TIMEOUT,
+// drains its own TMA loads and MMAs, releases TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <climits>
 #include <mutex>
 
 #include "fpx_internal.h"
@@ -26,13 +44,34 @@
 namespace fpx {
 namespace sm100 {
 
-constexpr int kTileM = 128;                 // query rows per tile (= block)
-constexpr int kTileN = 128;                 // keys per tile (= block)
+constexpr int kTileM = 128;   // query rows per tile (= block)
+constexpr int kTileN = 128;   // keys per block
 constexpr int kHeadDim = 128;
-constexpr int kThreads = 128;
-constexpr uint32_t kTileBytesMax = 32768;   // one 128 x 128 bf16 tile
-constexpr uint32_t kTmemCols = 256;         // S/P: columns [0, 128), O: [128, 256)
-constexpr size_t kSmemBytes = 5 * kTileBytesMax + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxRegs = 208;  // 256 x 208 + 128 x 64 <= 384 x 168 (registers at launch)
+constexpr int kOtherRegs = 64;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr uint32_t kSlotBytes = 32768;  // one 128 x 128 bf16 tile
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;    // lazy rescale threshold (log2 units)
+// shared memory: Q0, Q1, K slot 0/1, V slot 0/1 (32 KB each), then barriers
+constexpr uint32_t kOffQ = 0, kOffK = 2 * kSlotBytes, kOffV = 4 * kSlotBytes,
+                   kOffBar = 6 * kSlotBytes;
+constexpr size_t kSmemBytes = 6 * kSlotBytes + 256 + 1024;
+
+enum Bar {
+  kBarQ = 0,
+  kBarKFull = 1,    // +slot
+  kBarKEmpty = 3,   // +slot
+  kBarVFull = 5,    // +slot
+  kBarVEmpty = 7,   // +slot
+  kBarSFull = 9,    // +tile
+  kBarPReady = 11,  // +tile
+  kBarODone = 13,   // +tile
+  kBarDrain = 15,
+  kNumBars = 16
+};
 
 template <bool kFp8>
 struct Cfg {
@@ -41,9 +80,8 @@ struct Cfg {
   static constexpr uint32_t kBoxBytes = 128 * 128;                   // 128 rows x 128 B
   static constexpr int kBoxes = kTileBytes / kBoxBytes;              // 1 or 2 (along D)
   static constexpr int kKStep = kFp8 ? 32 : 16;                      // MMA K per instruction
-  static constexpr int kQKSteps = kHeadDim / kKStep;                 // 4 or 8
-  static constexpr int kPVSteps = kTileN / kKStep;                   // 4 or 8
-  static constexpr int kPCols = kTileN * kElem / 4;                  // P columns in TMEM
+  static constexpr int kQKSteps = kHeadDim / kKStep;
+  static constexpr int kPVSteps = kTileN / kKStep;
   static constexpr uint32_t kIdescQK = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, false, 128, 128);
   static constexpr uint32_t kIdescPV = make_idesc(kFp8 ? 0 : 1, kFp8 ? 0 : 1, true, 128, 128);
 };
@@ -52,8 +90,134 @@ struct Cfg {
 // kBoxes boxes of [128 rows x 128 B].
 template <bool kFp8>
 __device__ __forceinline__ uint32_t kmajor_koff(int kk) {
-  constexpr int per_box = 128 / (Cfg<kFp8>::kKStep * Cfg<kFp8>::kElem);  // k-steps per 128 B
+  constexpr int per_box = 128 / (Cfg<kFp8>::kKStep * Cfg<kFp8>::kElem);
   return (kk / per_box) * Cfg<kFp8>::kBoxBytes + (kk % per_box) * 32;
+}
+
+// Union of two CSR rows, consumed in list order.  Every entry of each row is visited exactly
+// once; entries outside [0, I] are skipped.  With ascending rows (as fpx_select writes them) the
+// union is ascending and shared blocks are visited once for both tiles.
+struct RowMerge {
+  const int32_t* ci;
+  int a, a_end, b, b_end, I;
+  __device__ __forceinline__ bool ok(int J) const { return J >= 0 && J <= I; }
+  __device__ __forceinline__ bool next(int& J, int& uses) {
+    while (a < a_end && !ok(ci[a])) ++a;
+    while (b < b_end && !ok(ci[b])) ++b;
+    if (a >= a_end && b >= b_end) return false;
+    const int ja = a < a_end ? ci[a] : INT_MAX;
+    const int jb = b < b_end ? ci[b] : INT_MAX;
+    J = min(ja, jb);
+    uses = (ja == J ? 1 : 0) | (jb == J ? 2 : 0);
+    if (ja == J) ++a;
+    if (jb == J) ++b;
+    return true;
+  }
+};
+
+// Maximum of 128 fp32 values (3-input max, eight independent chains).
+__device__ __forceinline__ float row_max128(const uint32_t* r) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = __uint_as_float(r[k]);
+#pragma unroll
+  for (int j = 8; j < 128; j += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      m[k] = max3f(m[k], __uint_as_float(r[j + k]), __uint_as_float(r[j + 8 + k]));
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// 2^x on the FMA pipe, for x <= 128 (x below -126 flushes towards 0).  Cody-Waite style split
+// x = n + f, n = round(x) via the 1.5 * 2^23 shifter (the low bits of t then hold n), |f| <= 1/2;
+// 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative error on
+// [-1/2, 1/2] (Remez exchange; fitted by exp2_poly_fit.py, max relative error 7.5e-5, below
+// bf16 and e4m3 rounding of P); 2^n is added in the exponent field.
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f;
+  constexpr float C2 = 0.2426111251115799f, C3 = 0.0551716685295105f;
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0 = x0, t1 = x1, kShift, kShift);
+  fadd2(n0 = t0, n1 = t1, -kShift, -kShift);
+  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
+  ffma2(p0, p1, C3, C3, f0, f1, C2, C2);
+  ffma2(p0, p1, p0, p1, f0, f1, C1, C1);
+  ffma2(p0, p1, p0, p1, f0, f1, C0, C0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// One in kPolyEvery element pairs takes exp2 on the FMA pipe instead of the MUFU (0: none), to
+// balance the two pipes.
+#ifndef FPX_POLY_EVERY
+#define FPX_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FPX_POLY_EVERY;
+
+// r[0..127] holds a row of S (fp32 bits); on return r holds P packed for the P*V MMA (bf16
+// pairs in r[0..63], or e4m3 quads in r[0..31]) and the row sum of P is returned.
+template <bool kFp8>
+__device__ __forceinline__ float softmax_row_to_p(uint32_t* r, float sl2, float neg_m) {
+  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 128; j += 2) {
+    float x0, x1, p0, p1;
+    ffma2(x0, x1, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), sl2, sl2, neg_m, neg_m);
+    constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
+    if (kPolyEvery > 0 && (j / 2) % kEvery == kEvery - 1) {
+      exp2_poly2(p0, p1, x0, x1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    fadd2(s[(j / 2) % 4 * 2], s[(j / 2) % 4 * 2 + 1], p0, p1);
+    if (kFp8) {
+      // four consecutive keys per 32-bit column: low half now, high half at j % 4 == 2
+      const uint32_t v = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+      if ((j & 2) == 0) r[j / 4] = v;
+      else r[j / 4] |= v << 16;
+    } else {
+      r[j / 2] = pack_bf16x2(p0, p1);
+    }
+  }
+  return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+}
+
+struct Unit {
+  int kvh, b, s, I, tok0, n_s, ntiles;
+  int h[2], r[2], beg[2], end[2];
+};
+
+__device__ __forceinline__ Unit decode_unit(const ProblemDesc& p, const int32_t* blk_base,
+                                            const int32_t* row_ptr, int u) {
+  Unit w;
+  const int pairs = (p.group + 1) / 2;
+  const int per_kv = p.nb_total * pairs;
+  w.kvh = u / per_kv;
+  const int rem = u - w.kvh * per_kv;
+  w.b = rem / pairs;
+  const int pair = rem - w.b * pairs;
+  w.s = seq_of_block(blk_base, p.num_seqs, w.b);
+  w.I = w.b - blk_base[w.s];
+  w.tok0 = seq_start(p, w.s);
+  w.n_s = seq_len(p, w.s);
+  w.ntiles = (2 * pair + 1 < p.group) ? 2 : 1;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    w.h[t] = w.kvh * p.group + 2 * pair + t;
+    if (t < w.ntiles) {
+      w.r[t] = w.h[t] * p.nb_total + w.b;
+      w.beg[t] = row_ptr[w.r[t]];
+      w.end[t] = row_ptr[w.r[t] + 1];
+    } else {
+      w.r[t] = -1;
+      w.beg[t] = w.end[t] = 0;
+    }
+  }
+  return w;
 }
 
 template <bool kFp8>
@@ -61,51 +225,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, ProblemDesc p,
                const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-               __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-               SeqTables tab, const int32_t* __restrict__ order, StatusBlock* st) {
+               __nv_bfloat16* __restrict__ o, float* __restrict__ lse, SeqTables tab,
+               const int32_t* __restrict__ order, StatusBlock* st) {
   using C = Cfg<kFp8>;
   if (!*tab.valid) return;  // inconsistent cu_seqlens (recorded by the plan kernel)
-  const int32_t* __restrict__ blk_base = tab.blk_base;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - raw_u32);
-  const uint32_t sQ = sbase;
-  // stage x: K at sK0 + x * kTileBytesMax, V at sV0 + x * kTileBytesMax
-  const uint32_t sK0 = sbase + kTileBytesMax, sV0 = sbase + 3 * kTileBytesMax;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + 5 * kTileBytesMax);
-  const uint32_t bar_q = smem_u32(&bars[0]);
-  const uint32_t bar_kv0 = smem_u32(&bars[1]);  // stage x: bar_kv0 + 8 * x
-  const uint32_t bar_mma = smem_u32(&bars[3]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[4]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[5]);
+  const uint32_t bar0 = sbase + kOffBar;  // barrier i at bar0 + 8 * i
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 8 * kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * kNumBars + 4);
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-
-  // ---- tile coordinates -------------------------------------------------------------------
-  const int r = order ? order[blockIdx.x] : blockIdx.x;
-  const int h = r / p.nb_total;
-  const int b = r - h * p.nb_total;
-  const int s = seq_of_block(blk_base, p.num_seqs, b);
-  const int I = b - blk_base[s];
-  const int n_s = seq_len(p, s);
-  const int tok0 = seq_start(p, s);
-  const int kvh = h / p.group;
-  const int q_tok = tok0 + I * kTileM;
-  const int beg = row_ptr[r], end = row_ptr[r + 1];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Unit w = decode_unit(p, tab.blk_base, row_ptr, order ? order[blockIdx.x] : blockIdx.x);
 
   if (tid == 0) {
-    mbar_init(bar_q, 1);
-    mbar_init(bar_kv0, 1);
-    mbar_init(bar_kv0 + 8, 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(bar(kBarQ), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarKFull + i), 1);
+      mbar_init(bar(kBarKEmpty + i), 1);
+      mbar_init(bar(kBarVFull + i), 1);
+      mbar_init(bar(kBarVEmpty + i), 1);
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarPReady + i), kTileM);
+      mbar_init(bar(kBarODone + i), 1);
+    }
+    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -113,220 +264,282 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem, tO = tmem + 128;
-
-  // TMA loads in flight (thread 0's bookkeeping, used to drain them on an aborted tile)
-  int kv_issued0 = 0, kv_issued1 = 0, kv_waited0 = 0, kv_waited1 = 0;
-  bool q_issued = false, q_waited = false;
-
-  // Loads the K/V tiles of key block J into stage `stg` (thread 0 only).
-  auto issue_kv = [&](int J, int stg) {
-    const int kv_tok = tok0 + J * kTileN;
-    if (stg) ++kv_issued1; else ++kv_issued0;
-    const uint32_t bar = bar_kv0 + 8 * stg;
-    mbar_arrive_expect_tx(bar, 2 * C::kTileBytes);
+  if (warp >= 8) {
+  setmaxnreg_dec<kOtherRegs>();
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------------ TMA producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
+      RowMerge peek = m;
+      int J, uses;
+      int n = 0;
+      bool q_issued = false;
+      if (peek.next(J, uses)) {
+        q_issued = true;
+        mbar_arrive_expect_tx(bar(kBarQ), C::kTileBytes * w.ntiles);
 #pragma unroll
-    for (int bx = 0; bx < C::kBoxes; ++bx) {
-      tma_load_3d(sK0 + stg * kTileBytesMax + bx * C::kBoxBytes, &tmK, bar, bx * 128 / C::kElem, kvh, kv_tok);
-      tma_load_3d(sV0 + stg * kTileBytesMax + bx * C::kBoxBytes, &tmV, bar, bx * 128 / C::kElem, kvh, kv_tok);
-    }
-  };
-  auto valid_J = [&](int J) { return J >= 0 && J <= I; };
-
-  // next valid entry at or after e (all threads compute the same sequence)
-  auto next_valid = [&](int e) {
-    while (e < end && !valid_J(col_idx[e])) ++e;
-    return e;
-  };
-
-  int e = next_valid(beg);
-  if (tid == 0) {
-    for (int x = beg; x < end; ++x)
-      if (!valid_J(col_idx[x])) { record_error(st, FPX_ERR_DEVICE_INPUT, 30, r, col_idx[x]); break; }
-    if (e < end) {
-      q_issued = true;
-      mbar_arrive_expect_tx(bar_q, C::kTileBytes);
+        for (int t = 0; t < 2; ++t) {
+          if (t >= w.ntiles) break;
 #pragma unroll
-      for (int bx = 0; bx < C::kBoxes; ++bx)
-        tma_load_3d(sQ + bx * C::kBoxBytes, &tmQ, bar_q, bx * 128 / C::kElem, h, q_tok);
-      issue_kv(col_idx[e], 0);
-    }
-  }
-
-  float sl2 = p.scale * 1.4426950408889634f;
-  float vsc = 1.f;
-  if (kFp8) {
-    sl2 *= p.q_scale[h] * p.k_scale[kvh];
-    vsc = p.v_scale[kvh];
-  }
-  const int my_row = tid;  // TMEM lane == query row of this thread
-  float m_run = -CUDART_INF_F, l_run = 0.f;
-  uint32_t mma_phase = 0;
-  int it = 0;
-  bool ok = true;
-
-  while (e < end && ok) {
-    const int J = col_idx[e];
-    const int stg = it & 1;
-    const int e_next = next_valid(e + 1);
-    if (tid == 0) {
-      if (e_next < end) issue_kv(col_idx[e_next], stg ^ 1);
-      bool good = true;
-      if (it == 0) good = q_waited = mbar_wait(bar_q, 0, abort_flag);
-      if (good) {
-        good = mbar_wait(bar_kv0 + 8 * stg, (it >> 1) & 1, abort_flag);
-        if (good) { if (stg) ++kv_waited1; else ++kv_waited0; }
-      }
-      if (good) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::kQKSteps; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sQ + kmajor_koff<kFp8>(kk), 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK0 + stg * kTileBytesMax + kmajor_koff<kFp8>(kk), 16, 1024);
-          if (kFp8) mma_f8_ss(tS, ad, bd, C::kIdescQK, kk > 0);
-          else mma_f16_ss(tS, ad, bd, C::kIdescQK, kk > 0);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(sbase + kOffQ + t * kSlotBytes + bx * C::kBoxBytes, &tmQ, bar(kBarQ),
+                        bx * 128 / C::kElem, w.h[t], w.tok0 + w.I * kTileM);
         }
-        mma_commit(bar_mma);
-      } else {
+      }
+      while (m.next(J, uses)) {
+        const int slot = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        const int kv_tok = w.tok0 + J * kTileN;
+        if (!mbar_wait(bar(kBarKEmpty + slot), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(kBarKFull + slot), C::kTileBytes);
+#pragma unroll
+        for (int bx = 0; bx < C::kBoxes; ++bx)
+          tma_load_3d(sbase + kOffK + slot * kSlotBytes + bx * C::kBoxBytes, &tmK,
+                      bar(kBarKFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
+        if (!mbar_wait(bar(kBarVEmpty + slot), ph ^ 1, abort_flag)) {
+          // K of this entry is in flight; only its K barrier is drained below
+          volatile int never = 0;
+          mbar_wait(bar(kBarKFull + slot), ph, &never);
+          break;
+        }
+        mbar_arrive_expect_tx(bar(kBarVFull + slot), C::kTileBytes);
+#pragma unroll
+        for (int bx = 0; bx < C::kBoxes; ++bx)
+          tma_load_3d(sbase + kOffV + slot * kSlotBytes + bx * C::kBoxBytes, &tmV,
+                      bar(kBarVFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
+        ++n;
+      }
+      // Drain: wait (bounded) until every load this thread issued has landed.  On the normal
+      // path each of these has already completed.
+      volatile int never = 0;
+      if (q_issued) mbar_wait(bar(kBarQ), 0, &never);
+      for (int k = n - 2; k < n; ++k) {
+        if (k < 0) continue;
+        const int slot = k & 1;
+        const uint32_t ph = (k >> 1) & 1;
+        mbar_wait(bar(kBarKFull + slot), ph, &never);
+        mbar_wait(bar(kBarVFull + slot), ph, &never);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer -------
+    if (lane == 0) {
+      RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
+      int J_next = 0, uses_next = 0;
+      bool have_next = m.next(J_next, uses_next);
+      int u_next = 0;                    // union index of the next S to issue
+      int pv_pending0 = -1, pv_pending1 = -1;  // union index whose P*V is still to be issued
+      uint32_t p_phase0 = 0, p_phase1 = 0;
+      int o_started0 = 0, o_started1 = 0;
+      int v_users0 = 0, v_users1 = 0;
+      bool ok = true;
+      if (have_next) ok = mbar_wait(bar(kBarQ), 0, abort_flag);
+      uint64_t t_idle = 0;
+      // issues O_t += P_t V for the pending union entry n of tile t if P_t and V are ready
+      auto try_pv = [&](int t, int& pending, uint32_t& p_phase, int& o_started) -> bool {
+        if (pending < 0) return false;
+        const int n = pending;
+        const int slot = n & 1;
+        if (!mbar_try_wait(bar(kBarPReady + t), p_phase)) return false;
+        if (!mbar_try_wait(bar(kBarVFull + slot), (n >> 1) & 1)) return false;
+        p_phase ^= 1;
+        tc_fence_after();
+        const uint32_t vbase = sbase + kOffV + slot * kSlotBytes;
+#pragma unroll
+        for (int kk = 0; kk < C::kPVSteps; ++kk) {
+          const uint64_t bd = smem_desc_sw128(vbase + kk * C::kKStep * 128, 16384, 1024);
+          const uint32_t acc = (o_started || kk > 0) ? 1u : 0u;
+          if (kFp8)
+            mma_f8_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bd, C::kIdescPV, acc);
+          else
+            mma_f16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bd, C::kIdescPV, acc);
+        }
+        o_started = 1;
+        const int left = slot ? --v_users1 : --v_users0;
+        if (left == 0) mma_commit(bar(kBarVEmpty + slot));
+        pending = -1;
+        return true;
+      };
+      while (ok && (have_next || pv_pending0 >= 0 || pv_pending1 >= 0)) {
+        bool progressed = try_pv(0, pv_pending0, p_phase0, o_started0);
+        progressed |= try_pv(1, pv_pending1, p_phase1, o_started1);
+        if (have_next) {
+          const bool u0 = uses_next & 1, u1 = (uses_next >> 1) & 1;
+          const int slot = u_next & 1;
+          // The slot's previous entry must have issued all its P*V reads of V before the
+          // slot's reader count is reset for this entry.
+          const int users_left = slot ? v_users1 : v_users0;
+          if ((!u0 || pv_pending0 < 0) && (!u1 || pv_pending1 < 0) && users_left == 0 &&
+              mbar_try_wait(bar(kBarKFull + slot), (u_next >> 1) & 1)) {
+            tc_fence_after();
+            const uint32_t kbase = sbase + kOffK + slot * kSlotBytes;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!((uses_next >> t) & 1)) continue;
+              const uint32_t qbase = sbase + kOffQ + t * kSlotBytes;
+#pragma unroll
+              for (int kk = 0; kk < C::kQKSteps; ++kk) {
+                const uint64_t ad = smem_desc_sw128(qbase + kmajor_koff<kFp8>(kk), 16, 1024);
+                const uint64_t bd = smem_desc_sw128(kbase + kmajor_koff<kFp8>(kk), 16, 1024);
+                if (kFp8) mma_f8_ss(tmem + t * 128, ad, bd, C::kIdescQK, kk > 0);
+                else mma_f16_ss(tmem + t * 128, ad, bd, C::kIdescQK, kk > 0);
+              }
+              mma_commit(bar(kBarSFull + t));
+              if (t == 0) pv_pending0 = u_next; else pv_pending1 = u_next;
+            }
+            mma_commit(bar(kBarKEmpty + slot));
+            if (slot) v_users1 = (u0 ? 1 : 0) + (u1 ? 1 : 0);
+            else v_users0 = (u0 ? 1 : 0) + (u1 ? 1 : 0);
+            ++u_next;
+            have_next = m.next(J_next, uses_next);
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_idle = 0;
+        } else {
+          if (*abort_flag) ok = false;
+          const uint64_t now = globaltimer_ns();
+          if (t_idle == 0) t_idle = now;
+          else if (now - t_idle > kWaitLimitNs) ok = false;
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      mma_commit(bar(kBarODone + 0));
+      mma_commit(bar(kBarODone + 1));
+      // drain: every MMA issued by this thread completes before TMEM can be released
+      mma_commit(bar(kBarDrain));
+      volatile int never = 0;
+      mbar_wait(bar(kBarDrain), 0, &never);
+    }
+  }
+  } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
+    // ------------------------------------------------------------------ softmax ----------
+    const int t = warp >> 2;                 // tile
+    const int row = tid & 127;               // query row = TMEM lane
+    const int my_h = t ? w.h[1] : w.h[0];
+    const int my_r = t ? w.r[1] : w.r[0];
+    const int my_beg = t ? w.beg[1] : w.beg[0];
+    const int my_end = t ? w.end[1] : w.end[0];
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t * 128 + lane_base;
+    const uint32_t tO = tmem + 256 + t * 128 + lane_base;
+    const int qpos = w.I * kTileM + row;
+    const bool write = t < w.ntiles && qpos < w.n_s;
+    const int64_t tq = static_cast<int64_t>(w.tok0) + qpos;
+    float sl2 = p.scale * 1.4426950408889634f;
+    float vsc = 1.f;
+    if (kFp8 && t < w.ntiles) {
+      sl2 *= p.q_scale[my_h] * p.k_scale[w.kvh];
+      vsc = p.v_scale[w.kvh];
+    }
+    float m_ref = -CUDART_INF_F, l_run = 0.f;
+    uint32_t s_phase = 0;
+    int it = 0;
+    bool ok = true;
+    if (t < w.ntiles) {
+      for (int e = my_beg; e < my_end; ++e) {
+        const int J = col_idx[e];
+        if (J < 0 || J > w.I) {
+          if (row == 0) record_error(st, FPX_ERR_DEVICE_INPUT, 30, my_r, J);
+          continue;
+        }
+        if (!mbar_wait(bar(kBarSFull + t), s_phase, abort_flag)) { ok = false; break; }
+        s_phase ^= 1;
+        tc_fence_after();
+        const bool diag = (J == w.I);
+        // the whole S row of this thread: 128 fp32 in registers (one TMEM read)
+        uint32_t r[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, r + c * 32);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_wait_ld(r + c * 32);
+        if (diag) {  // token causal mask: key column > query row
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
+        }
+        const float mx = row_max128(r) * sl2;  // finite: key 0 is visible to every row
+        // lazy rescale: move the reference max only when the block max exceeds it by > 2^8
+        float corr = 1.f;
+        if (mx > m_ref + kRescaleLog2) {
+          corr = ex2_approx(m_ref - mx);  // 0 for the first block
+          l_run *= corr;
+          m_ref = mx;
+        }
+        if (it > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+          // O_t is stable: the previous P*V into it completed before S_t was written
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_wait_ld(ov);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * corr);
+            tmem_st32(tO + c * 32, ov);
+          }
+        }
+        // P = exp2(s * sl2 - m_ref), packed in place and written over S
+        const float rs = softmax_row_to_p<kFp8>(r, sl2, -m_ref);
+        if (kFp8) {
+          tmem_st32(tS, r);
+        } else {
+          tmem_st32(tS, r);
+          tmem_st32(tS + 32, r + 32);
+        }
+        l_run += rs;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPReady + t));
+        ++it;
+      }
+      // epilogue: wait for the last P*V, normalise, store O (bf16) and the natural-log LSE
+      if (ok && it > 0 && !mbar_wait(bar(kBarODone + t), 0, abort_flag)) ok = false;
+      if (!ok) {
         *abort_flag = 1;
+        if (row == 0) record_error(st, FPX_ERR_TIMEOUT, 31, my_r, it);
+      } else {
+        tc_fence_after();
+        uint4* orow = reinterpret_cast<uint4*>(o + (tq * p.hq + my_h) * kHeadDim);
+        if (it == 0) {
+          if (write) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
+            if (lse) lse[static_cast<int64_t>(my_h) * p.total_tokens + tq] = -CUDART_INF_F;
+          }
+        } else {
+          const float inv = vsc / l_run;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_wait_ld(r);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 v4;
+              v4.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+              v4.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+              v4.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+              v4.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+              if (write) orow[c * 4 + i] = v4;
+            }
+          }
+          if (lse && write)
+            lse[static_cast<int64_t>(my_h) * p.total_tokens + tq] =
+                (m_ref + __log2f(l_run)) * 0.6931471805599453f;
+        }
       }
     }
-    if (!mbar_wait(bar_mma, mma_phase, abort_flag)) { ok = false; break; }
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // ---- softmax on this thread's row ------------------------------------------------------
-    uint32_t sr[128];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_base + c * 32, sr + c * 32);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_wait_ld(sr + c * 32);
-    float x[128];
-    float mx = -CUDART_INF_F;
-    const bool diag = (J == I);
-#pragma unroll
-    for (int j = 0; j < 128; ++j) {
-      float v = __uint_as_float(sr[j]) * sl2;
-      if (diag && j > my_row) v = -CUDART_INF_F;
-      x[j] = v;
-      mx = fmaxf(mx, v);
-    }
-    const float m_new = fmaxf(m_run, mx);  // finite: key 0 of the block is always visible
-    const float corr = ex2_approx(m_run - m_new);
-    // Rescale O rows whose max moved (the previous P*V has completed).  tcgen05.ld/st are
-    // warp-collective, so the whole warp takes the branch; rows that did not move scale by 1.
-    if (it > 0 && __any_sync(0xffffffffu, m_new > m_run)) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t orow[32];
-        tmem_ld32(tO + lane_base + c * 32, orow);
-        tmem_wait_ld(orow);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * corr);
-        tmem_st32(tO + lane_base + c * 32, orow);
-      }
-    }
-    float psum = 0.f;
-    uint32_t pk[64];
-    if (kFp8) {
-#pragma unroll
-      for (int j = 0; j < 128; j += 4) {
-        const float p0 = ex2_approx(x[j] - m_new), p1 = ex2_approx(x[j + 1] - m_new);
-        const float p2 = ex2_approx(x[j + 2] - m_new), p3 = ex2_approx(x[j + 3] - m_new);
-        psum += (p0 + p1) + (p2 + p3);
-        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
-        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
-        pk[j / 4] = lo | (hi << 16);
-      }
-      tmem_st32(tS + lane_base, pk);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 128; j += 2) {
-        const float p0 = ex2_approx(x[j] - m_new), p1 = ex2_approx(x[j + 1] - m_new);
-        psum += p0 + p1;
-        pk[j / 2] = pack_bf16x2(p0, p1);
-      }
-      tmem_st32(tS + lane_base, pk);
-      tmem_st32(tS + lane_base + 32, pk + 32);
-    }
-    l_run = l_run * corr + psum;
-    m_run = m_new;
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < C::kPVSteps; ++kk) {
-        const uint32_t voff = kk * C::kKStep * 128;  // kKStep key rows of 128 B
-        const uint64_t bd = smem_desc_sw128(sV0 + stg * kTileBytesMax + voff, 16384, 1024);
-        if (kFp8) mma_f8_ts(tO, tS + kk * 8, bd, C::kIdescPV, (it > 0 || kk > 0));
-        else mma_f16_ts(tO, tS + kk * 8, bd, C::kIdescPV, (it > 0 || kk > 0));
-      }
-      mma_commit(bar_mma);
-    }
-    if (!mbar_wait(bar_mma, mma_phase, abort_flag)) { ok = false; break; }
-    mma_phase ^= 1;
-    tc_fence_after();
-    e = e_next;
-    ++it;
   }
 
-  if (!ok) {
-    if (tid == 0) record_error(st, FPX_ERR_TIMEOUT, 31, r, it);
-    *abort_flag = 1;
-  }
-
-  // ---- epilogue -------------------------------------------------------------------------------
-  // `ok` and `it` are uniform across the CTA, so every warp executes the (warp-collective) TMEM
-  // loads together; only the global stores depend on the row.
-  const int qpos = I * kTileM + my_row;
-  const bool write = qpos < n_s;
-  const int64_t tq = static_cast<int64_t>(tok0) + qpos;
-  uint4* orow = reinterpret_cast<uint4*>(o + (tq * p.hq + h) * kHeadDim);
-  if (ok && it == 0) {
-    if (write) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
-      if (lse) lse[static_cast<int64_t>(h) * p.total_tokens + tq] = -CUDART_INF_F;
-    }
-  } else if (ok) {
-    const float inv = vsc / l_run;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t ov[32];
-      tmem_ld32(tO + lane_base + c * 32, ov);
-      tmem_wait_ld(ov);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]) * inv, __uint_as_float(ov[8 * i + 1]) * inv);
-        w.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]) * inv, __uint_as_float(ov[8 * i + 3]) * inv);
-        w.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]) * inv, __uint_as_float(ov[8 * i + 5]) * inv);
-        w.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]) * inv, __uint_as_float(ov[8 * i + 7]) * inv);
-        if (write) orow[c * 4 + i] = w;
-      }
-    }
-    if (lse && write)
-      lse[static_cast<int64_t>(h) * p.total_tokens + tq] =
-          (m_run + __log2f(l_run)) * 0.6931471805599453f;
-  }
-
-  // ---- teardown: never release TMEM while an MMA may still be writing it ----------------------
-  if (!ok && tid == 0) {
-    // drain: bounded waits for this tile's own TMA loads still in flight and for a committed
-    // MMA, so that neither writes shared memory or TMEM after the CTA has released them
-    volatile int never = 0;
-    if (q_issued && !q_waited) mbar_wait(bar_q, 0, &never);
-    if (kv_issued0 > kv_waited0) mbar_wait(bar_kv0, (kv_issued0 - 1) & 1, &never);
-    if (kv_issued1 > kv_waited1) mbar_wait(bar_kv0 + 8, (kv_issued1 - 1) & 1, &never);
-    mbar_wait(bar_mma, mma_phase, &never);
-  }
+  // ---- teardown: every role has drained its own async work ------------------------------
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -370,14 +583,18 @@ bool attn_tc_supported(const ProblemDesc& p, fpx_dtype dt) {
   return (dt == FPX_BF16 || dt == FPX_E4M3) && p.d == 128 && p.block == 128;
 }
 
+int64_t attn_tc_units(const ProblemDesc& p) {
+  return static_cast<int64_t>(p.hkv) * p.nb_total * ((p.group + 1) / 2);
+}
+
 cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                            const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                            void* o, float* lse, SeqTables t, const int32_t* order,
                            StatusBlock* st, cudaStream_t s, bool* encode_failed) {
   using namespace sm100;
   *encode_failed = false;
-  const int R = p.hq * p.nb_total;
-  if (R == 0) return cudaSuccess;
+  const int64_t units = attn_tc_units(p);
+  if (units == 0) return cudaSuccess;
   const bool fp8 = dt == FPX_E4M3;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, p.total_tokens, p.hq, p.d, fp8) ||
@@ -390,8 +607,8 @@ cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, co
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  kern<<<R, kThreads, kSmemBytes, s>>>(mq, mk, mv, p, row_ptr, col_idx,
-                                       static_cast<__nv_bfloat16*>(o), lse, t, order, st);
+  kern<<<static_cast<unsigned>(units), kThreads, kSmemBytes, s>>>(
+      mq, mk, mv, p, row_ptr, col_idx, static_cast<__nv_bfloat16*>(o), lse, t, order, st);
   return cudaGetLastError();
 }
 

@@ -23,7 +23,9 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
                           SeqTables t, StatusBlock* st, cudaStream_t s);
 
 // fpx_sparse_prefill: tile schedule, then one of the two attention kernels.
-cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, cudaStream_t s);
+// `units`: schedule the tensor-core kernel's two-head units instead of single CSR rows.
+cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, bool units,
+                         cudaStream_t s);
 cudaError_t launch_attn_simt(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              void* o, float* lse, SeqTables t, const int32_t* order,

@@ -482,19 +482,34 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
 }
 
 // ------------------------------------------------------------------------------------------
-// order: the attention tile schedule.  Rows are grouped by KV head (so the CTAs resident at
-// any moment share K/V blocks through L2) and, inside a group, heaviest first (largest local
-// block index I first, since a row can keep at most I + 1 blocks), then sequence, then head.
-//   pos(h, s, I) = kvh*g*NB + g*sum_s' max(0, nb_s' - 1 - I) + g*#{s' < s : nb_s' > I} + h%g
+// order: the attention schedule.  Items are grouped by KV head (so the CTAs resident at any
+// moment share K/V blocks through L2) and, inside a group, heaviest first (largest local block
+// index I first, since a row can keep at most I + 1 blocks), then sequence, then slot:
+//   pos = kvh*slots*NB + slots*sum_s' max(0, nb_s' - 1 - I) + slots*#{s' < s : nb_s' > I} + sub
+// Rows (CUDA-core kernel): item r = h*NB + b, slots = Hq/Hkv, sub = h % slots.
+// Units (tensor-core kernel, two Q heads of one KV group): item u = (kvh*NB + b)*slots + sub
+// with slots = ceil((Hq/Hkv) / 2), sub = the head pair.
 // ------------------------------------------------------------------------------------------
 __global__ void order_kernel(ProblemDesc p, const int32_t* __restrict__ blk_base,
-                             const int32_t* __restrict__ valid, int32_t* __restrict__ order) {
+                             const int32_t* __restrict__ valid, int32_t* __restrict__ order,
+                             int units) {
   if (!*valid) return;
-  const int R = p.hq * p.nb_total;
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= R) return;
-  const int h = r / p.nb_total;
-  const int b = r - h * p.nb_total;
+  const int slots = units ? (p.group + 1) / 2 : p.group;
+  const int n_items = p.hkv * p.nb_total * slots;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_items) return;
+  int kvh, b, sub;
+  if (units) {
+    kvh = i / (p.nb_total * slots);
+    const int rem = i - kvh * p.nb_total * slots;
+    b = rem / slots;
+    sub = rem - b * slots;
+  } else {
+    const int h = i / p.nb_total;
+    b = i - h * p.nb_total;
+    kvh = h / p.group;
+    sub = h - kvh * p.group;
+  }
   const int s = seq_of_block(blk_base, p.num_seqs, b);
   const int I = b - blk_base[s];
   int64_t heavier = 0, same_earlier = 0;
@@ -503,16 +518,17 @@ __global__ void order_kernel(ProblemDesc p, const int32_t* __restrict__ blk_base
     heavier += max(0, nb2 - 1 - I);
     if (s2 < s && nb2 > I) ++same_earlier;
   }
-  const int g = p.group, kvh = h / g;
-  const int64_t pos = static_cast<int64_t>(kvh) * g * p.nb_total + g * heavier +
-                      g * same_earlier + (h % g);
-  order[pos] = r;
+  const int64_t pos = static_cast<int64_t>(kvh) * slots * p.nb_total + slots * heavier +
+                      slots * same_earlier + sub;
+  order[pos] = i;
 }
 
-cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, cudaStream_t s) {
-  const int R = p.hq * p.nb_total;
-  if (R == 0) return cudaSuccess;
-  order_kernel<<<(R + 255) / 256, 256, 0, s>>>(p, t.blk_base, t.valid, order);
+cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, bool units,
+                         cudaStream_t s) {
+  const int slots = units ? (p.group + 1) / 2 : p.group;
+  const int n_items = p.hkv * p.nb_total * slots;
+  if (n_items == 0) return cudaSuccess;
+  order_kernel<<<(n_items + 255) / 256, 256, 0, s>>>(p, t.blk_base, t.valid, order, units ? 1 : 0);
   return cudaGetLastError();
 }
 
