@@ -10,21 +10,24 @@
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for tile 0: one query row (= one TMEM lane) per thread
 //   warps 4-7  softmax for tile 1
-//   warp  8    tcgen05.mma issue (one thread), TMEM allocation
-//   warp  9    TMA loads (one thread): Q0/Q1 once, then K_J and V_J into 2-slot rings
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warp  8    tcgen05.mma issue for tile 0 (one elected lane), TMEM allocation
+//   warp  9    tcgen05.mma issue for tile 1
+//   warp  10   TMA loads (one elected lane): Q0/Q1 once, then K_J and V_J into 2-slot rings
+//   warp  11   idle (completes the third warpgroup)
 // setmaxnreg moves registers from the third warpgroup to the two softmax warpgroups, which
 // hold a whole 128-column S row in registers.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_t (bf16 / e4m3)
 // is written over the first columns of S_t and read from TMEM by the P*V MMA.
 //
-// Per kept block the MMA thread issues S_t = Q_t K_J^T, and later O_t += P_t V_J as soon as
-// softmax t has published P_t.  It never waits on one operation while another is ready (it
-// polls K arrivals and both tiles' P barriers), so a tile that skips blocks never stalls the
-// other one and every ring slot is released as soon as its last reader is issued.  S_t for
-// the next block is issued only after O_t += P_t V for the previous one (P aliases S), so when
-// softmax t sees S_t complete, the previous P*V into O_t has completed too and O_t may be
-// rescaled in place.
+// The tensor pipe buffers only a few MMA instructions, so an issuing thread that stops to wait
+// or to do bookkeeping starves it.  Each tile therefore has its own issuing warp running a plain
+// sequential loop over the union of the two rows: S_t(n) = Q_t K_n^T, wait for softmax t to
+// publish P_t(n), O_t += P_t(n) V_n, next block.  While one warp waits for its softmax, the other
+// warp's MMAs keep the tensor pipe busy (ping-pong).  Because a warp issues S_t(n + 1) after
+// O_t += P_t(n) V_n, the completion of S_t(n + 1) (tracked by that warp's commit) implies the
+// previous P*V into O_t has completed, so softmax t may rescale O_t in place.  Both issuing warps
+// release every ring slot they pass (a commit after their MMAs, or a plain arrive for blocks their
+// tile does not use), so the slot barriers count one arrival per tile.
 //
 // Softmax: exp2 domain, lazy rescale (the reference max only moves when the block max exceeds it
 // by more than 2^8), two passes over S in TMEM (row max, then P) so that only 32 columns are live
@@ -48,10 +51,10 @@ constexpr int kTileM = 128;   // query rows per tile (= block)
 constexpr int kTileN = 128;   // keys per block
 constexpr int kHeadDim = 128;
 constexpr int kThreads = 384;
-constexpr int kSoftmaxRegs = 208;  // 256 x 208 + 128 x 64 <= 384 x 168 (registers at launch)
-constexpr int kOtherRegs = 64;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kSoftmaxRegs = 208;  // 256 x 208 + 128 x 80 <= 384 x 168 (registers at launch)
+constexpr int kOtherRegs = 80;
+constexpr int kMmaWarp0 = 8;   // issues tile 0's MMAs; warp 9 issues tile 1's
+constexpr int kLoadWarp = 10;
 constexpr uint32_t kSlotBytes = 32768;  // one 128 x 128 bf16 tile
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;    // lazy rescale threshold (log2 units)
@@ -69,8 +72,8 @@ enum Bar {
   kBarSFull = 9,    // +tile
   kBarPReady = 11,  // +tile
   kBarODone = 13,   // +tile
-  kBarDrain = 15,
-  kNumBars = 16
+  kBarDrain = 15,   // +tile
+  kNumBars = 17
 };
 
 template <bool kFp8>
@@ -238,25 +241,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * kNumBars + 4);
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const Unit w = decode_unit(p, tab.blk_base, row_ptr, order ? order[blockIdx.x] : blockIdx.x);
 
   if (tid == 0) {
     mbar_init(bar(kBarQ), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarKFull + i), 1);
-      mbar_init(bar(kBarKEmpty + i), 1);
+      mbar_init(bar(kBarKEmpty + i), w.ntiles);
       mbar_init(bar(kBarVFull + i), 1);
-      mbar_init(bar(kBarVEmpty + i), 1);
+      mbar_init(bar(kBarVEmpty + i), w.ntiles);
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarPReady + i), kTileM);
       mbar_init(bar(kBarODone + i), 1);
     }
-    mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDrain + 0), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -268,17 +272,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   setmaxnreg_dec<kOtherRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer ----
-    if (lane == 0) {
+    // Warp-uniform loop; one elected lane issues the copies.
+    constexpr unsigned kFull = 0xffffffffu;
+    if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
-      RowMerge peek = m;
-      int J, uses;
-      int n = 0;
-      bool q_issued = false;
-      if (peek.next(J, uses)) {
-        q_issued = true;
+    }
+    RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
+    RowMerge peek = m;
+    int J, uses;
+    int n = 0;
+    bool q_issued = false;
+    if (peek.next(J, uses)) {
+      q_issued = true;
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(kBarQ), C::kTileBytes * w.ntiles);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -289,131 +297,119 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         bx * 128 / C::kElem, w.h[t], w.tok0 + w.I * kTileM);
         }
       }
-      while (m.next(J, uses)) {
-        const int slot = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        const int kv_tok = w.tok0 + J * kTileN;
-        if (!mbar_wait(bar(kBarKEmpty + slot), ph ^ 1, abort_flag)) break;
+    }
+    while (m.next(J, uses)) {
+      const int slot = n & 1;
+      const uint32_t ph = (n >> 1) & 1;
+      const int kv_tok = w.tok0 + J * kTileN;
+      if (!__all_sync(kFull, mbar_wait(bar(kBarKEmpty + slot), ph ^ 1, abort_flag))) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(kBarKFull + slot), C::kTileBytes);
 #pragma unroll
         for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_3d(sbase + kOffK + slot * kSlotBytes + bx * C::kBoxBytes, &tmK,
                       bar(kBarKFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
-        if (!mbar_wait(bar(kBarVEmpty + slot), ph ^ 1, abort_flag)) {
-          // K of this entry is in flight; only its K barrier is drained below
-          volatile int never = 0;
-          mbar_wait(bar(kBarKFull + slot), ph, &never);
-          break;
-        }
+      }
+      if (!__all_sync(kFull, mbar_wait(bar(kBarVEmpty + slot), ph ^ 1, abort_flag))) {
+        // K of this entry is in flight; only its K barrier is drained below
+        volatile int never = 0;
+        mbar_wait(bar(kBarKFull + slot), ph, &never);
+        break;
+      }
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(kBarVFull + slot), C::kTileBytes);
 #pragma unroll
         for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_3d(sbase + kOffV + slot * kSlotBytes + bx * C::kBoxBytes, &tmV,
                       bar(kBarVFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
-        ++n;
       }
-      // Drain: wait (bounded) until every load this thread issued has landed.  On the normal
-      // path each of these has already completed.
-      volatile int never = 0;
-      if (q_issued) mbar_wait(bar(kBarQ), 0, &never);
-      for (int k = n - 2; k < n; ++k) {
-        if (k < 0) continue;
-        const int slot = k & 1;
-        const uint32_t ph = (k >> 1) & 1;
-        mbar_wait(bar(kBarKFull + slot), ph, &never);
-        mbar_wait(bar(kBarVFull + slot), ph, &never);
-      }
+      ++n;
     }
-  } else if (warp == kMmaWarp) {
+    // Drain: wait (bounded) until every load this warp issued has landed.  On the normal path
+    // each of these has already completed.
+    volatile int never = 0;
+    if (q_issued) mbar_wait(bar(kBarQ), 0, &never);
+    for (int k = n - 2; k < n; ++k) {
+      if (k < 0) continue;
+      const int slot = k & 1;
+      const uint32_t ph = (k >> 1) & 1;
+      mbar_wait(bar(kBarKFull + slot), ph, &never);
+      mbar_wait(bar(kBarVFull + slot), ph, &never);
+    }
+  } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
     // ------------------------------------------------------------------ MMA issuer -------
-    if (lane == 0) {
+    // One warp per tile, warp-uniform sequential loop; one elected lane issues and commits.
+    constexpr unsigned kFull = 0xffffffffu;
+    const int t = warp - kMmaWarp0;
+    if (t < w.ntiles) {
+      // Matrix descriptors of every buffer, built once.  A k-step inside a buffer only moves the
+      // start-address field (bits 0-13, address >> 4): a constant add to the descriptor.
+      const uint64_t qdesc = smem_desc_sw128(sbase + kOffQ + t * kSlotBytes, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, 16384, 1024);
+      constexpr uint64_t kSlotDesc = kSlotBytes >> 4;
+      const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
       RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
-      int J_next = 0, uses_next = 0;
-      bool have_next = m.next(J_next, uses_next);
-      int u_next = 0;                    // union index of the next S to issue
-      int pv_pending0 = -1, pv_pending1 = -1;  // union index whose P*V is still to be issued
-      uint32_t p_phase0 = 0, p_phase1 = 0;
-      int o_started0 = 0, o_started1 = 0;
-      int v_users0 = 0, v_users1 = 0;
+      RowMerge peek = m;
+      int J, uses;
       bool ok = true;
-      if (have_next) ok = mbar_wait(bar(kBarQ), 0, abort_flag);
-      uint64_t t_idle = 0;
-      // issues O_t += P_t V for the pending union entry n of tile t if P_t and V are ready
-      auto try_pv = [&](int t, int& pending, uint32_t& p_phase, int& o_started) -> bool {
-        if (pending < 0) return false;
-        const int n = pending;
+      if (peek.next(J, uses)) ok = __all_sync(kFull, mbar_wait(bar(kBarQ), 0, abort_flag));
+      uint32_t p_phase = 0;
+      bool o_started = false;
+      int n = 0;
+      while (ok && m.next(J, uses)) {
         const int slot = n & 1;
-        if (!mbar_try_wait(bar(kBarPReady + t), p_phase)) return false;
-        if (!mbar_try_wait(bar(kBarVFull + slot), (n >> 1) & 1)) return false;
-        p_phase ^= 1;
-        tc_fence_after();
-        const uint32_t vbase = sbase + kOffV + slot * kSlotBytes;
-#pragma unroll
-        for (int kk = 0; kk < C::kPVSteps; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vbase + kk * C::kKStep * 128, 16384, 1024);
-          const uint32_t acc = (o_started || kk > 0) ? 1u : 0u;
-          if (kFp8)
-            mma_f8_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bd, C::kIdescPV, acc);
-          else
-            mma_f16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bd, C::kIdescPV, acc);
-        }
-        o_started = 1;
-        const int left = slot ? --v_users1 : --v_users0;
-        if (left == 0) mma_commit(bar(kBarVEmpty + slot));
-        pending = -1;
-        return true;
-      };
-      while (ok && (have_next || pv_pending0 >= 0 || pv_pending1 >= 0)) {
-        bool progressed = try_pv(0, pv_pending0, p_phase0, o_started0);
-        progressed |= try_pv(1, pv_pending1, p_phase1, o_started1);
-        if (have_next) {
-          const bool u0 = uses_next & 1, u1 = (uses_next >> 1) & 1;
-          const int slot = u_next & 1;
-          // The slot's previous entry must have issued all its P*V reads of V before the
-          // slot's reader count is reset for this entry.
-          const int users_left = slot ? v_users1 : v_users0;
-          if ((!u0 || pv_pending0 < 0) && (!u1 || pv_pending1 < 0) && users_left == 0 &&
-              mbar_try_wait(bar(kBarKFull + slot), (u_next >> 1) & 1)) {
+        const uint32_t ph = (n >> 1) & 1;
+        const bool mine = (uses >> t) & 1;
+        if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + slot), ph, abort_flag))) { ok = false; break; }
+        if (elect_one()) {
+          if (mine) {
             tc_fence_after();
-            const uint32_t kbase = sbase + kOffK + slot * kSlotBytes;
+            const uint64_t kdesc = dk0 + slot * kSlotDesc;
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (!((uses_next >> t) & 1)) continue;
-              const uint32_t qbase = sbase + kOffQ + t * kSlotBytes;
-#pragma unroll
-              for (int kk = 0; kk < C::kQKSteps; ++kk) {
-                const uint64_t ad = smem_desc_sw128(qbase + kmajor_koff<kFp8>(kk), 16, 1024);
-                const uint64_t bd = smem_desc_sw128(kbase + kmajor_koff<kFp8>(kk), 16, 1024);
-                if (kFp8) mma_f8_ss(tmem + t * 128, ad, bd, C::kIdescQK, kk > 0);
-                else mma_f16_ss(tmem + t * 128, ad, bd, C::kIdescQK, kk > 0);
-              }
-              mma_commit(bar(kBarSFull + t));
-              if (t == 0) pv_pending0 = u_next; else pv_pending1 = u_next;
+            for (int kk = 0; kk < C::kQKSteps; ++kk) {
+              const uint64_t off = kmajor_koff<kFp8>(kk) >> 4;
+              if (kFp8) mma_f8_ss(tS, qdesc + off, kdesc + off, C::kIdescQK, kk > 0);
+              else mma_f16_ss(tS, qdesc + off, kdesc + off, C::kIdescQK, kk > 0);
             }
+            mma_commit(bar(kBarSFull + t));
             mma_commit(bar(kBarKEmpty + slot));
-            if (slot) v_users1 = (u0 ? 1 : 0) + (u1 ? 1 : 0);
-            else v_users0 = (u0 ? 1 : 0) + (u1 ? 1 : 0);
-            ++u_next;
-            have_next = m.next(J_next, uses_next);
-            progressed = true;
+          } else {
+            mbar_arrive(bar(kBarKEmpty + slot));
           }
         }
-        if (progressed) {
-          t_idle = 0;
-        } else {
-          if (*abort_flag) ok = false;
-          const uint64_t now = globaltimer_ns();
-          if (t_idle == 0) t_idle = now;
-          else if (now - t_idle > kWaitLimitNs) ok = false;
+        if (mine) {
+          if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + t), p_phase, abort_flag))) { ok = false; break; }
+          p_phase ^= 1;
         }
+        if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + slot), ph, abort_flag))) { ok = false; break; }
+        if (elect_one()) {
+          if (mine) {
+            tc_fence_after();
+            const uint64_t vdesc = dv0 + slot * kSlotDesc;
+#pragma unroll
+            for (int kk = 0; kk < C::kPVSteps; ++kk) {
+              const uint32_t acc = (o_started || kk > 0) ? 1u : 0u;
+              const uint64_t bd = vdesc + ((kk * C::kKStep * 128) >> 4);
+              if (kFp8) mma_f8_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
+              else mma_f16_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
+            }
+            mma_commit(bar(kBarVEmpty + slot));
+          } else {
+            mbar_arrive(bar(kBarVEmpty + slot));
+          }
+        }
+        if (mine) o_started = true;
+        ++n;
       }
       if (!ok) *abort_flag = 1;
-      mma_commit(bar(kBarODone + 0));
-      mma_commit(bar(kBarODone + 1));
-      // drain: every MMA issued by this thread completes before TMEM can be released
-      mma_commit(bar(kBarDrain));
+      if (elect_one()) {
+        mma_commit(bar(kBarODone + t));
+        // drain: every MMA issued by this warp completes before TMEM can be released
+        mma_commit(bar(kBarDrain + t));
+      }
       volatile int never = 0;
-      mbar_wait(bar(kBarDrain), 0, &never);
+      mbar_wait(bar(kBarDrain + t), 0, &never);
     }
   }
   } else {
@@ -539,7 +535,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // ---- teardown: every role has drained its own async work ------------------------------
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
