@@ -82,8 +82,9 @@ size_t scratch_bytes(const fpx_problem* p, const Sizes& s, int which) {
     case 0:  // pooled Q and K, fp32
       return align_up(sizeof(float) * s.nb * p->hq * p->d, 256) +
              align_up(sizeof(float) * s.nb * p->hkv * p->d, 256);
-    case 1:  // row max, keep counts, overflow flag
-      return align_up(sizeof(float) * R, 256) + align_up(sizeof(int32_t) * R, 256) + 256;
+    case 1:  // row max, keep counts, per-CTA totals, overflow flag
+      return align_up(sizeof(float) * R, 256) + align_up(sizeof(int32_t) * R, 256) +
+             align_up(sizeof(int64_t) * (R / 8 + 1), 256) + 256;
     case 2:  // tile schedule
       return align_up(sizeof(int32_t) * R, 256);
     default:
@@ -210,15 +211,17 @@ fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, in
   char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
   float* rowmax = reinterpret_cast<float*>(scratch);
   int32_t* counts = reinterpret_cast<int32_t*>(scratch + align_up(sizeof(float) * R, 256));
-  int* overflow = reinterpret_cast<int*>(scratch + align_up(sizeof(float) * R, 256) +
-                                         align_up(sizeof(int32_t) * R, 256));
+  int64_t* cta_tot = reinterpret_cast<int64_t*>(scratch + align_up(sizeof(float) * R, 256) +
+                                                 align_up(sizeof(int32_t) * R, 256));
+  int* overflow = reinterpret_cast<int*>(reinterpret_cast<char*>(cta_tot) +
+                                         align_up(sizeof(int64_t) * (R / 8 + 1), 256));
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   // window / sink beyond any row are equivalent to "all": clamp so the device compare stays
   // in range
   const int sink = sink_blocks > d.nb_total ? d.nb_total + 1 : sink_blocks;
   const int window = window_blocks > d.nb_total ? d.nb_total + 1 : window_blocks;
   if (launch_select(d, scores, alpha, sink, window, row_ptr, col_idx, col_capacity, nnz_d, rowmax,
-                    counts, overflow, t, st, s) != cudaSuccess)
+                    counts, cta_tot, overflow, t, st, s) != cudaSuccess)
     return FPX_ERR_CUDA;
   return FPX_OK;
 }

@@ -19,8 +19,10 @@ cudaError_t launch_score(const ProblemDesc& p, fpx_dtype dt, const float* qbar, 
 // fpx_select: row max + keep count, scan into row_ptr, emit col_idx.
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
-                          int64_t* nnz_d, float* rowmax, int32_t* counts, int* overflow,
-                          SeqTables t, StatusBlock* st, cudaStream_t s);
+                          int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
+                          int* overflow, SeqTables t, StatusBlock* st, cudaStream_t s);
+// CTAs of the select kernels (each owns 8 rows); the workspace holds one int64 per CTA.
+int select_ctas(const ProblemDesc& p);
 
 // fpx_sparse_prefill: tile schedule, then one of the two attention kernels.
 // `units`: schedule the tensor-core kernel's two-head units instead of single CSR rows.

@@ -25,11 +25,13 @@ constexpr int kPlanThreads = 256;
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(ProblemDesc p, SeqTables t,
                                                             StatusBlock* st) {
-  __shared__ int64_t s_nb[kPlanThreads];
-  __shared__ int64_t s_tri[kPlanThreads];
-  __shared__ int s_bad[kPlanThreads];
+  __shared__ int64_t w_nb[kPlanThreads / 32], w_tri[kPlanThreads / 32];
+  __shared__ int s_bad;
   const int S = p.num_seqs;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  // contiguous chunk of sequences per thread
   const int per = (S + kPlanThreads - 1) / kPlanThreads;
   const int lo = min(S, tid * per), hi = min(S, lo + per);
   int64_t nb_sum = 0, tri_sum = 0;
@@ -41,23 +43,45 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(ProblemDesc p, SeqTa
     nb_sum += nb;
     tri_sum += nb * (nb + 1) / 2;
   }
-  s_nb[tid] = nb_sum;
-  s_tri[tid] = tri_sum;
-  s_bad[tid] = bad ? 1 : 0;
-  __syncthreads();
-  if (tid == 0) {  // exclusive scan of the per-thread sums (256 entries)
-    int64_t a = 0, b = 0;
-    for (int i = 0; i < kPlanThreads; ++i) {
-      const int64_t x = s_nb[i], y = s_tri[i];
-      s_nb[i] = a;
-      s_tri[i] = b;
+  if (bad) atomicOr(&s_bad, 1);
+  // block-wide exclusive scan of (nb_sum, tri_sum): warp shuffles, then across warps
+  int64_t a = nb_sum, b = tri_sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
       a += x;
       b += y;
     }
-    bool good = true;
-    for (int i = 0; i < kPlanThreads; ++i) good = good && s_bad[i] == 0;
+  }
+  if (lane == 31) {
+    w_nb[wid] = a;
+    w_tri[wid] = b;
+  }
+  __syncthreads();
+  int64_t base_nb = 0, base_tri = 0, tot_nb = 0, tot_tri = 0;
+#pragma unroll
+  for (int i = 0; i < kPlanThreads / 32; ++i) {
+    if (i < wid) {
+      base_nb += w_nb[i];
+      base_tri += w_tri[i];
+    }
+    tot_nb += w_nb[i];
+    tot_tri += w_tri[i];
+  }
+  int64_t nb_run = base_nb + a - nb_sum, tri_run = base_tri + b - tri_sum;
+  for (int s = lo; s < hi; ++s) {
+    const int n = seq_len(p, s);
+    const int64_t nb = n > 0 ? (n + p.block - 1) / p.block : 0;
+    t.blk_base[s] = static_cast<int32_t>(nb_run);
+    t.tri_base[s] = tri_run;
+    nb_run += nb;
+    tri_run += nb * (nb + 1) / 2;
+  }
+  if (tid == 0) {
+    bool good = s_bad == 0;
     if (!good) record_error(st, FPX_ERR_DEVICE_INPUT, 3);
-    if (a != p.nb_total || b != p.tri_total) {
+    if (tot_nb != p.nb_total || tot_tri != p.tri_total) {
       record_error(st, FPX_ERR_DEVICE_INPUT, 1);
       good = false;
     }
@@ -68,18 +92,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(ProblemDesc p, SeqTa
     // Every later kernel of the stage returns at once unless the tables are consistent with
     // the sizes the host used for the grids and the caller used for the buffers.
     *t.valid = good ? 1 : 0;
-    t.blk_base[S] = static_cast<int32_t>(a);
-    t.tri_base[S] = b;
-  }
-  __syncthreads();
-  int64_t nb_run = s_nb[tid], tri_run = s_tri[tid];
-  for (int s = lo; s < hi; ++s) {
-    const int n = seq_len(p, s);
-    const int64_t nb = n > 0 ? (n + p.block - 1) / p.block : 0;
-    t.blk_base[s] = static_cast<int32_t>(nb_run);
-    t.tri_base[s] = tri_run;
-    nb_run += nb;
-    tri_run += nb * (nb + 1) / 2;
+    t.blk_base[S] = static_cast<int32_t>(tot_nb);
+    t.tri_base[S] = tot_tri;
   }
 }
 
@@ -210,9 +224,9 @@ cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const
 }
 
 // ------------------------------------------------------------------------------------------
-// score: one CTA per (64 consecutive global query blocks, Q head).  It walks the 64-wide key
-// tiles from the first block of the earliest sequence it touches up to its diagonal tile; a
-// pair (b, c) of global blocks is written iff both lie in the same sequence and c <= b.
+// score: one CTA per (64 x 64 tile of global block pairs (b, c) with c <= b, Q head); the tiles
+// of the lower triangle are enumerated by blockIdx.x.  A pair is written iff both blocks lie in
+// the same sequence and c <= b; tiles that hold no such pair return at once.
 // ------------------------------------------------------------------------------------------
 constexpr int kScoreTile = 64;
 constexpr int kScoreThreads = 256;  // 16 x 16 threads, 4 x 4 outputs each
@@ -229,82 +243,70 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ProblemDesc p,
   extern __shared__ float4 score_smem[];
   float* sq = reinterpret_cast<float*>(score_smem);  // [D][64] (transposed)
   float* sk = sq + D * kScoreTile;                   // [D][64]
+  // lower-triangle tile index -> (x, y), y <= x
+  const int k = blockIdx.x;
+  int x = static_cast<int>((sqrtf(8.f * k + 1.f) - 1.f) * 0.5f);
+  while (x * (x + 1) / 2 > k) --x;
+  while ((x + 1) * (x + 2) / 2 <= k) ++x;
+  const int y = k - x * (x + 1) / 2;
   const int h = blockIdx.y;
   const int kvh = h / p.group;
-  const int b0 = blockIdx.x * kScoreTile;
+  const int b0 = x * kScoreTile, c0 = y * kScoreTile;
   const int b_last = min(p.nb_total, b0 + kScoreTile) - 1;
+  // key tiles left of the first sequence this query tile touches hold no valid pair
+  const int first_col = blk_base[seq_of_block(blk_base, p.num_seqs, b0)];
+  if (c0 + kScoreTile <= first_col) return;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   float scale = p.scale;
   if (p.q_scale) scale *= p.q_scale[h] * p.k_scale[kvh];
 
-  // query tile (transposed into [d][row])
+  // consecutive threads take consecutive rows, so the transposed shared-memory stores below
+  // hit consecutive banks
   for (int i = tid; i < kScoreTile * (D / 4); i += kScoreThreads) {
-    const int row = i / (D / 4), c4 = (i % (D / 4)) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int row = i % kScoreTile, c4 = (i / kScoreTile) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f), u = v;
     if (b0 + row <= b_last)
       v = *reinterpret_cast<const float4*>(qbar + (static_cast<int64_t>(b0 + row) * p.hq + h) * D + c4);
+    if (c0 + row < p.nb_total)
+      u = *reinterpret_cast<const float4*>(kbar + (static_cast<int64_t>(c0 + row) * p.hkv + kvh) * D + c4);
     sq[(c4 + 0) * kScoreTile + row] = v.x;
     sq[(c4 + 1) * kScoreTile + row] = v.y;
     sq[(c4 + 2) * kScoreTile + row] = v.z;
     sq[(c4 + 3) * kScoreTile + row] = v.w;
+    sk[(c4 + 0) * kScoreTile + row] = u.x;
+    sk[(c4 + 1) * kScoreTile + row] = u.y;
+    sk[(c4 + 2) * kScoreTile + row] = u.z;
+    sk[(c4 + 3) * kScoreTile + row] = u.w;
   }
-  // per-row metadata for the 4 rows this thread writes
-  int row_seq[4], row_first[4];
-  int64_t row_base[4];
+  __syncthreads();
+  float acc[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int b = b0 + ty * 4 + i;
-    if (b <= b_last) {
-      const int s = seq_of_block(blk_base, p.num_seqs, b);
-      const int I = b - blk_base[s];
-      row_seq[i] = s;
-      row_first[i] = blk_base[s];
-      row_base[i] = static_cast<int64_t>(h) * p.tri_total + tri_base[s] +
-                    static_cast<int64_t>(I) * (I + 1) / 2 - blk_base[s];
-    } else {
-      row_seq[i] = -1;
-      row_first[i] = 0;
-      row_base[i] = 0;
-    }
-  }
-  const int first_col = blk_base[seq_of_block(blk_base, p.num_seqs, b0)];
-  for (int c0 = (first_col / kScoreTile) * kScoreTile; c0 <= b_last; c0 += kScoreTile) {
-    __syncthreads();
-    for (int i = tid; i < kScoreTile * (D / 4); i += kScoreThreads) {
-      const int col = i / (D / 4), c4 = (i % (D / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + col < p.nb_total)
-        v = *reinterpret_cast<const float4*>(kbar + (static_cast<int64_t>(c0 + col) * p.hkv + kvh) * D + c4);
-      sk[(c4 + 0) * kScoreTile + col] = v.x;
-      sk[(c4 + 1) * kScoreTile + col] = v.y;
-      sk[(c4 + 2) * kScoreTile + col] = v.z;
-      sk[(c4 + 3) * kScoreTile + col] = v.w;
-    }
-    __syncthreads();
-    float acc[4][4];
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+  for (int dd = 0; dd < D; ++dd) {
+    const float4 a = *reinterpret_cast<const float4*>(sq + dd * kScoreTile + ty * 4);
+    const float4 c = *reinterpret_cast<const float4*>(sk + dd * kScoreTile + tx * 4);
+    const float av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-    for (int dd = 0; dd < D; ++dd) {
-      const float4 a = *reinterpret_cast<const float4*>(sq + dd * kScoreTile + ty * 4);
-      const float4 c = *reinterpret_cast<const float4*>(sk + dd * kScoreTile + tx * 4);
-      const float av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], cv[j], acc[i][j]);
+  }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 4; ++i) {
+    const int b = b0 + ty * 4 + i;
+    if (b > b_last) continue;
+    const int s = seq_of_block(blk_base, p.num_seqs, b);
+    const int first = blk_base[s];
+    const int I = b - first;
+    const int64_t row_base = static_cast<int64_t>(h) * p.tri_total + tri_base[s] +
+                             static_cast<int64_t>(I) * (I + 1) / 2 - first;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], cv[j], acc[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (row_seq[i] < 0) continue;
-      const int b = b0 + ty * 4 + i;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = c0 + tx * 4 + j;
-        if (c >= row_first[i] && c <= b) scores[row_base[i] + c] = acc[i][j] * scale;
-      }
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c >= first && c <= b) scores[row_base + c] = acc[i][j] * scale;
     }
   }
 }
@@ -312,7 +314,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ProblemDesc p,
 cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, const float* kbar,
                          float* scores, SeqTables t, cudaStream_t s) {
   if (p.nb_total == 0) return cudaSuccess;
-  dim3 grid((p.nb_total + kScoreTile - 1) / kScoreTile, p.hq);
+  const int nt = (p.nb_total + kScoreTile - 1) / kScoreTile;
+  dim3 grid(nt * (nt + 1) / 2, p.hq);
   const size_t smem = 2 * sizeof(float) * p.d * kScoreTile;
   if (p.d == 128) {
     cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -327,9 +330,14 @@ cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, con
 }
 
 // ------------------------------------------------------------------------------------------
-// select: warp per row r = (h, s, I).
+// select: a CTA owns 8 consecutive rows r = (h, s, I) (warp per row).
+//   count: row max, kept-block count per row, CTA total
+//   scan:  exclusive scan of the CTA totals (one CTA), nnz, capacity check
+//   emit:  per-CTA exclusive scan of its counts -> row_ptr; ballot/popc compaction -> col_idx
 // ------------------------------------------------------------------------------------------
 constexpr int kSelWarps = 8;
+constexpr int kSelRowsPerWarp = 1;
+constexpr int kSelRows = kSelWarps * kSelRowsPerWarp;
 
 struct RowInfo {
   int64_t base;  // first score of the row
@@ -357,39 +365,64 @@ __device__ __forceinline__ bool keep_block(float score, float rowmax, float alph
   return expf(score - rowmax) >= alpha;
 }
 
-__global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
-    ProblemDesc p, const float* __restrict__ scores, float alpha, int sink, int window,
-    float* __restrict__ rowmax, int32_t* __restrict__ counts, SeqTables t) {
-  if (!*t.valid) return;
-  const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
-  const int R = p.hq * p.nb_total;
-  if (r >= R) return;
-  const RowInfo ri = row_info(p, t, r);
-  const float* row = scores + ri.base;
-  float m = -CUDART_INF_F;
-  for (int j = lane; j < ri.len; j += 32) m = fmaxf(m, __ldcs(row + j));
+__device__ __forceinline__ float row_max_warp(const float* __restrict__ row, int len, int lane) {
+  float m0 = -CUDART_INF_F, m1 = m0, m2 = m0, m3 = m0;
+  for (int j = lane; j < len; j += 128) {  // four independent loads in flight per lane
+    m0 = fmaxf(m0, __ldg(row + j));
+    if (j + 32 < len) m1 = fmaxf(m1, __ldg(row + j + 32));
+    if (j + 64 < len) m2 = fmaxf(m2, __ldg(row + j + 64));
+    if (j + 96 < len) m3 = fmaxf(m3, __ldg(row + j + 96));
+  }
+  float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  int cnt = 0;
-  for (int j0 = 0; j0 < ri.len; j0 += 32) {
-    const int j = j0 + lane;
-    const bool kp = j < ri.len && keep_block(row[j], m, alpha, j, ri.I, sink, window);
-    cnt += __popc(__ballot_sync(0xffffffffu, kp));
+  return m;
+}
+
+__global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
+    ProblemDesc p, const float* __restrict__ scores, float alpha, int sink, int window,
+    float* __restrict__ rowmax, int32_t* __restrict__ counts, int64_t* __restrict__ cta_tot,
+    SeqTables t) {
+  if (!*t.valid) return;
+  __shared__ int w_tot[kSelWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int R = p.hq * p.nb_total;
+  int tot = 0;
+  for (int k = 0; k < kSelRowsPerWarp; ++k) {
+    const int r = blockIdx.x * kSelRows + warp * kSelRowsPerWarp + k;
+    if (r >= R) break;
+    const RowInfo ri = row_info(p, t, r);
+    const float* row = scores + ri.base;
+    const float m = row_max_warp(row, ri.len, lane);
+    int cnt = 0;
+    for (int j0 = 0; j0 < ri.len; j0 += 32) {
+      const int j = j0 + lane;
+      const bool kp = j < ri.len && keep_block(row[j], m, alpha, j, ri.I, sink, window);
+      cnt += __popc(__ballot_sync(0xffffffffu, kp));
+    }
+    if (lane == 0) {
+      rowmax[r] = m;
+      counts[r] = cnt;
+    }
+    tot += cnt;
   }
-  if (lane == 0) {
-    rowmax[r] = m;
-    counts[r] = cnt;
+  if (lane == 0) w_tot[warp] = tot;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t a = 0;
+#pragma unroll
+    for (int i = 0; i < kSelWarps; ++i) a += w_tot[i];
+    cta_tot[blockIdx.x] = a;
   }
 }
 
 constexpr int kScanThreads = 1024;
 
-// Exclusive scan of counts into row_ptr (single CTA); nnz, capacity check.
+// Exclusive scan of the per-CTA totals (single CTA); nnz, row_ptr[R], capacity check.
 __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
-    int R, const int32_t* __restrict__ counts, int32_t* __restrict__ row_ptr, int64_t capacity,
-    int64_t* __restrict__ nnz_d, int* __restrict__ overflow, const int32_t* __restrict__ valid,
-    StatusBlock* st) {
+    int R, int nblk, int64_t* __restrict__ cta_tot, int32_t* __restrict__ row_ptr,
+    int64_t capacity, int64_t* __restrict__ nnz_d, int* __restrict__ overflow,
+    const int32_t* __restrict__ valid, StatusBlock* st) {
   __shared__ int64_t warp_tot[32];
   if (!*valid) {  // inconsistent cu_seqlens (already recorded): publish an empty CSR
     for (int i = threadIdx.x; i <= R; i += blockDim.x) row_ptr[i] = 0;
@@ -400,10 +433,10 @@ __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
     return;
   }
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int per = (R + kScanThreads - 1) / kScanThreads;
-  const int lo = min(R, tid * per), hi = min(R, lo + per);
+  const int per = (nblk + kScanThreads - 1) / kScanThreads;
+  const int lo = min(nblk, tid * per), hi = min(nblk, lo + per);
   int64_t sum = 0;
-  for (int i = lo; i < hi; ++i) sum += counts[i];
+  for (int i = lo; i < hi; ++i) sum += cta_tot[i];
   int64_t x = sum;  // inclusive warp scan
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -424,8 +457,9 @@ __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
   __syncthreads();
   int64_t run = x - sum + (w > 0 ? warp_tot[w - 1] : 0);
   for (int i = lo; i < hi; ++i) {
-    row_ptr[i] = static_cast<int32_t>(run);
-    run += counts[i];
+    const int64_t c = cta_tot[i];
+    cta_tot[i] = run;  // in place: exclusive offsets
+    run += c;
   }
   if (tid == kScanThreads - 1) {
     const int64_t total = warp_tot[31];
@@ -440,44 +474,69 @@ __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
 
 __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
     ProblemDesc p, const float* __restrict__ scores, float alpha, int sink, int window,
-    const float* __restrict__ rowmax, const int32_t* __restrict__ row_ptr,
+    const float* __restrict__ rowmax, const int32_t* __restrict__ counts,
+    const int64_t* __restrict__ cta_off, int32_t* __restrict__ row_ptr,
     int32_t* __restrict__ col_idx, const int* __restrict__ overflow, SeqTables t) {
-  if (*overflow || !*t.valid) return;
-  const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
+  if (!*t.valid) return;
+  __shared__ int32_t s_off[kSelRows];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int R = p.hq * p.nb_total;
-  if (r >= R) return;
-  const RowInfo ri = row_info(p, t, r);
-  const float* row = scores + ri.base;
-  const float m = rowmax[r];
-  int32_t out = row_ptr[r];
-  for (int j0 = 0; j0 < ri.len; j0 += 32) {
-    const int j = j0 + lane;
-    const bool kp = j < ri.len && keep_block(__ldcs(row + j), m, alpha, j, ri.I, sink, window);
-    const unsigned bal = __ballot_sync(0xffffffffu, kp);
-    if (kp) col_idx[out + __popc(bal & ((1u << lane) - 1u))] = j;
-    out += __popc(bal);
+  const int r0 = blockIdx.x * kSelRows;
+  static_assert(kSelRows <= 32, "one lane per row in the CTA-local scan");
+  if (warp == 0) {  // exclusive scan of this CTA's counts (one per lane)
+    const int c = (lane < kSelRows && r0 + lane < R) ? counts[r0 + lane] : 0;
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < kSelRows) s_off[lane] = x - c;
+  }
+  __syncthreads();
+  const int64_t base = cta_off[blockIdx.x];
+  if (threadIdx.x < kSelRows && r0 + threadIdx.x < R)
+    row_ptr[r0 + threadIdx.x] = static_cast<int32_t>(base + s_off[threadIdx.x]);
+  if (*overflow) return;
+  for (int k = 0; k < kSelRowsPerWarp; ++k) {
+    const int rl = warp * kSelRowsPerWarp + k;
+    const int r = r0 + rl;
+    if (r >= R) break;
+    const RowInfo ri = row_info(p, t, r);
+    const float* row = scores + ri.base;
+    const float m = rowmax[r];
+    int64_t out = base + s_off[rl];
+    for (int j0 = 0; j0 < ri.len; j0 += 32) {
+      const int j = j0 + lane;
+      const bool kp = j < ri.len && keep_block(__ldcs(row + j), m, alpha, j, ri.I, sink, window);
+      const unsigned bal = __ballot_sync(0xffffffffu, kp);
+      if (kp) col_idx[out + __popc(bal & ((1u << lane) - 1u))] = j;
+      out += __popc(bal);
+    }
   }
 }
 
+int select_ctas(const ProblemDesc& p) { return (p.hq * p.nb_total + kSelRows - 1) / kSelRows; }
+
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
-                          int64_t* nnz_d, float* rowmax, int32_t* counts, int* overflow,
-                          SeqTables t, StatusBlock* st, cudaStream_t s) {
+                          int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
+                          int* overflow, SeqTables t, StatusBlock* st, cudaStream_t s) {
   const int R = p.hq * p.nb_total;
+  const int nblk = select_ctas(p);
   if (R > 0) {
-    const int grid = (R + kSelWarps - 1) / kSelWarps;
-    select_count_kernel<<<grid, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
-                                                       counts, t);
+    select_count_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
+                                                       counts, cta_tot, t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  select_scan_kernel<<<1, kScanThreads, 0, s>>>(R, counts, row_ptr, capacity, nnz_d, overflow,
-                                                t.valid, st);
+  select_scan_kernel<<<1, kScanThreads, 0, s>>>(R, nblk, cta_tot, row_ptr, capacity, nnz_d,
+                                                overflow, t.valid, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || R == 0) return e;
-  select_emit_kernel<<<(R + kSelWarps - 1) / kSelWarps, kSelWarps * 32, 0, s>>>(
-      p, scores, alpha, sink, window, rowmax, row_ptr, col_idx, overflow, t);
+  select_emit_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
+                                                     counts, cta_tot, row_ptr, col_idx, overflow,
+                                                     t);
   return cudaGetLastError();
 }
 

@@ -159,7 +159,7 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
  *   fpx_select_noalloc_max_bytes() bytes (2 MiB), which every GPU that loads the library holds
  *   until the process exits.  The caller still owns scores, row_ptr, col_idx and nnz_d.
  *   Same arguments and results as fpx_select, without ws / ws_bytes.
- *   Limits: the problem's fpx_workspace_bytes(p, 1) must not exceed the array (about 260,000
+ *   Limits: the problem's fpx_workspace_bytes(p, 1) must not exceed the array (about 230,000
  *   query-block rows Hq * NB for a few sequences); larger problems return FPX_ERR_CAPACITY
  *   before anything is launched.  An invalid or unsupported problem returns FPX_ERR_INVALID_ARG.
  *   Device-side conditions are visible through the outputs: nnz > col_capacity means nothing was
