@@ -30,7 +30,7 @@ STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "misaligned po
 EXPORTS = ("fpx_num_blocks", "fpx_scores_elems", "fpx_rows", "fpx_max_nnz", "fpx_workspace_bytes",
            "fpx_clear_status", "fpx_query_status", "fpx_status_string", "fpx_block_scores",
            "fpx_select", "fpx_sparse_prefill", "fpx_attention_path", "fpx_select_noalloc",
-           "fpx_select_noalloc_max_bytes")
+           "fpx_select_noalloc_max_bytes", "fpx_diag_bounded_wait")
 
 
 class FpxError(RuntimeError):
@@ -87,6 +87,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fpx_select_noalloc.restype = ctypes.c_int
     lib.fpx_select_noalloc_max_bytes.argtypes = []
     lib.fpx_select_noalloc_max_bytes.restype = sz
+    lib.fpx_diag_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
+    lib.fpx_diag_bounded_wait.restype = ctypes.c_int
     _lib = lib
     return lib
 

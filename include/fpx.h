@@ -175,6 +175,15 @@ fpx_status fpx_select_noalloc(const fpx_problem* p, const float* scores, float a
                               fpx_stream_t stream);
 size_t fpx_select_noalloc_max_bytes(void);
 
+/*
+ * Diagnostic for failure detection (the paper has no counterpart).  Launches one CTA that waits,
+ * with the same bounded-wait loop the pipeline barriers of fpx_sparse_prefill use, on an
+ * mbarrier phase that nothing completes.  The wait gives up after limit_ns nanoseconds
+ * (0 < limit_ns <= 2e9) and records FPX_ERR_TIMEOUT in the status block of `ws` (any workspace,
+ * 256-byte aligned); the CUDA context stays usable.  Returns a launch status only.
+ */
+fpx_status fpx_diag_bounded_wait(void* ws, uint64_t limit_ns, fpx_stream_t stream);
+
 /* Which attention kernel fpx_sparse_prefill uses for this problem: 1 = the tcgen05/TMEM
  * tensor-core mainloop (bf16 / e4m3, B = 128, D = 128), 0 = the CUDA-core kernel (fp32 and the
  * remaining shapes). */
