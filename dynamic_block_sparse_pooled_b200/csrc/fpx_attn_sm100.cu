@@ -10,29 +10,29 @@
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for tile 0: one query row (= one TMEM lane) per thread
 //   warps 4-7  softmax for tile 1
-//   warp  8    tcgen05.mma issue for tile 0 (one elected lane), TMEM allocation
-//   warp  9    tcgen05.mma issue for tile 1
+//   warp  8    tcgen05.mma issue for both tiles (one elected lane), TMEM allocation
 //   warp  10   TMA loads (one elected lane): Q0/Q1 once, then K_J and V_J into 2-slot rings
-//   warp  11   idle (completes the third warpgroup)
+//   warps 9, 11 idle (complete the third warpgroup)
 // setmaxnreg moves registers from the third warpgroup to the two softmax warpgroups, which
 // hold a whole 128-column S row in registers.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_t (bf16 / e4m3)
 // is written over the first columns of S_t and read from TMEM by the P*V MMA.
 //
-// The tensor pipe buffers only a few MMA instructions, so an issuing thread that stops to wait
-// or to do bookkeeping starves it.  Each tile therefore has its own issuing warp running a plain
-// sequential loop over the union of the two rows: S_t(n) = Q_t K_n^T, wait for softmax t to
-// publish P_t(n), O_t += P_t(n) V_n, next block.  While one warp waits for its softmax, the other
-// warp's MMAs keep the tensor pipe busy (ping-pong).  Because a warp issues S_t(n + 1) after
-// O_t += P_t(n) V_n, the completion of S_t(n + 1) (tracked by that warp's commit) implies the
-// previous P*V into O_t has completed, so softmax t may rescale O_t in place.  Both issuing warps
-// release every ring slot they pass (a commit after their MMAs, or a plain arrive for blocks their
-// tile does not use), so the slot barriers count one arrival per tile.
+// The tensor pipe buffers only a few MMA instructions, so the issuing thread must never stop for
+// long between groups.  One warp issues every MMA in a fixed order per union entry n:
+//     S_0(n) = Q_0 K_n^T | O_1 += P_1(n') V_n' | S_1(n) = Q_1 K_n^T | O_0 += P_0(n) V_n
+// where n' is tile 1's previous entry.  Softmax 0 of entry n then runs while the pipe executes
+// tile 1's P*V and S, and softmax 1 while it executes tile 0's P*V and next S, so the two
+// softmaxes alternate on the MUFU instead of contending for it.  S_t of an entry is always
+// issued after the previous O_t += P_t V (same thread, in-order pipe), so when softmax t sees S_t
+// complete, O_t is stable and may be rescaled in place.  Each ring slot is released by one commit
+// after the last MMA that reads it.
 //
 // Softmax: exp2 domain, lazy rescale (the reference max only moves when the block max exceeds it
-// by more than 2^8), two passes over S in TMEM (row max, then P) so that only 32 columns are live
-// in registers at a time.  Every wait is bounded: a broken pipeline records FPX_ERR_TIMEOUT,
-// drains its own TMA loads and MMAs, releases TMEM and exits.
+// by more than 2^8), the S row read from TMEM in two halves (the second in flight while the first
+// is reduced) and P written back in two halves (the first while the second is computed).  Every
+// wait is bounded: a broken pipeline records FPX_ERR_TIMEOUT, drains its own TMA loads and MMAs,
+// releases TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -53,7 +53,7 @@ constexpr int kHeadDim = 128;
 constexpr int kThreads = 384;
 constexpr int kSoftmaxRegs = 208;  // 256 x 208 + 128 x 80 <= 384 x 168 (registers at launch)
 constexpr int kOtherRegs = 80;
-constexpr int kMmaWarp0 = 8;   // issues tile 0's MMAs; warp 9 issues tile 1's
+constexpr int kMmaWarp = 8;    // issues every MMA; allocates TMEM
 constexpr int kLoadWarp = 10;
 constexpr uint32_t kSlotBytes = 32768;  // one 128 x 128 bf16 tile
 constexpr uint32_t kTmemCols = 512;
@@ -72,8 +72,8 @@ enum Bar {
   kBarSFull = 9,    // +tile
   kBarPReady = 11,  // +tile
   kBarODone = 13,   // +tile
-  kBarDrain = 15,   // +tile
-  kNumBars = 17
+  kBarDrain = 15,
+  kNumBars = 16
 };
 
 template <bool kFp8>
@@ -118,17 +118,18 @@ struct RowMerge {
   }
 };
 
-// Maximum of 128 fp32 values (3-input max, eight independent chains).
-__device__ __forceinline__ float row_max128(const uint32_t* r) {
-  float m[8];
+// Maximum of 64 fp32 values (3-input max, four independent chains).
+__device__ __forceinline__ float row_max64(const uint32_t* r) {
+  float m[4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m[k] = __uint_as_float(r[k]);
+  for (int k = 0; k < 4; ++k) m[k] = __uint_as_float(r[k]);
 #pragma unroll
-  for (int j = 8; j < 128; j += 16)
+  for (int j = 4; j < 60; j += 8)
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      m[k] = max3f(m[k], __uint_as_float(r[j + k]), __uint_as_float(r[j + 8 + k]));
-  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+    for (int k = 0; k < 4; ++k)
+      m[k] = max3f(m[k], __uint_as_float(r[j + k]), __uint_as_float(r[j + 4 + k]));
+  return max3f(max3f(m[0], m[1], __uint_as_float(r[60])), max3f(m[2], m[3], __uint_as_float(r[61])),
+               fmaxf(__uint_as_float(r[62]), __uint_as_float(r[63])));
 }
 
 // 2^x on the FMA pipe, for x <= 128 (x below -126 flushes towards 0).  Cody-Waite style split
@@ -153,20 +154,22 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// One in kPolyEvery element pairs takes exp2 on the FMA pipe instead of the MUFU (0: none), to
-// balance the two pipes.
+// One in kPolyEvery element pairs takes exp2 on the FMA pipe instead of the MUFU (0: none).  The
+// MUFU issues four ex2 per cycle per SM sub-partition, so a 128-column row costs ~1000 cycles
+// there; moving a quarter of the pairs to the FMA pipe was measured fastest (one in two or three
+// saturates the FMA pipe instead).
 #ifndef FPX_POLY_EVERY
-#define FPX_POLY_EVERY 0
+#define FPX_POLY_EVERY 4
 #endif
 constexpr int kPolyEvery = FPX_POLY_EVERY;
 
-// r[0..127] holds a row of S (fp32 bits); on return r holds P packed for the P*V MMA (bf16
-// pairs in r[0..63], or e4m3 quads in r[0..31]) and the row sum of P is returned.
-template <bool kFp8>
-__device__ __forceinline__ float softmax_row_to_p(uint32_t* r, float sl2, float neg_m) {
+// Columns [J0, J0 + 64) of the S row in r become P, packed in place (bf16 pairs at r[J0 / 2 ..],
+// or e4m3 quads at r[J0 / 4 ..]); returns their sum.
+template <bool kFp8, int J0>
+__device__ __forceinline__ float softmax_half_to_p(uint32_t* r, float sl2, float neg_m) {
   float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int j = 0; j < 128; j += 2) {
+  for (int j = J0; j < J0 + 64; j += 2) {
     float x0, x1, p0, p1;
     ffma2(x0, x1, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), sl2, sl2, neg_m, neg_m);
     constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
@@ -178,7 +181,6 @@ __device__ __forceinline__ float softmax_row_to_p(uint32_t* r, float sl2, float 
     }
     fadd2(s[(j / 2) % 4 * 2], s[(j / 2) % 4 * 2 + 1], p0, p1);
     if (kFp8) {
-      // four consecutive keys per 32-bit column: low half now, high half at j % 4 == 2
       const uint32_t v = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
       if ((j & 2) == 0) r[j / 4] = v;
       else r[j / 4] |= v << 16;
@@ -248,19 +250,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(bar(kBarQ), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarKFull + i), 1);
-      mbar_init(bar(kBarKEmpty + i), w.ntiles);
+      mbar_init(bar(kBarKEmpty + i), 1);
       mbar_init(bar(kBarVFull + i), 1);
-      mbar_init(bar(kBarVEmpty + i), w.ntiles);
+      mbar_init(bar(kBarVEmpty + i), 1);
       mbar_init(bar(kBarSFull + i), 1);
-      mbar_init(bar(kBarPReady + i), kTileM);
+      mbar_init(bar(kBarPReady + i), kTileM / 32);  // one arrival per softmax warp
       mbar_init(bar(kBarODone + i), 1);
     }
-    mbar_init(bar(kBarDrain + 0), 1);
-    mbar_init(bar(kBarDrain + 1), 1);
+    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -336,81 +337,119 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(bar(kBarKFull + slot), ph, &never);
       mbar_wait(bar(kBarVFull + slot), ph, &never);
     }
-  } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer -------
-    // One warp per tile, warp-uniform sequential loop; one elected lane issues and commits.
+    // Warp-uniform sequential loop; one elected lane issues and commits.  Order per union entry
+    // n:  S_0(n) | O_1 += P_1(n') V_n' (tile 1's previous entry) | S_1(n) | O_0 += P_0(n) V_n.
+    // Softmax 0 of entry n runs while the tensor pipe executes tile 1's P*V and S, and softmax 1
+    // while it executes tile 0's P*V and next S, so the two softmaxes alternate.
     constexpr unsigned kFull = 0xffffffffu;
-    const int t = warp - kMmaWarp0;
-    if (t < w.ntiles) {
-      // Matrix descriptors of every buffer, built once.  A k-step inside a buffer only moves the
-      // start-address field (bits 0-13, address >> 4): a constant add to the descriptor.
-      const uint64_t qdesc = smem_desc_sw128(sbase + kOffQ + t * kSlotBytes, 16, 1024);
-      const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, 16384, 1024);
-      constexpr uint64_t kSlotDesc = kSlotBytes >> 4;
-      const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
-      RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
-      RowMerge peek = m;
-      int J, uses;
-      bool ok = true;
-      if (peek.next(J, uses)) ok = __all_sync(kFull, mbar_wait(bar(kBarQ), 0, abort_flag));
-      uint32_t p_phase = 0;
-      bool o_started = false;
-      int n = 0;
-      while (ok && m.next(J, uses)) {
-        const int slot = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        const bool mine = (uses >> t) & 1;
-        if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + slot), ph, abort_flag))) { ok = false; break; }
-        if (elect_one()) {
-          if (mine) {
-            tc_fence_after();
-            const uint64_t kdesc = dk0 + slot * kSlotDesc;
+    // Matrix descriptors of every buffer, built once.  A k-step inside a buffer only moves the
+    // start-address field (bits 0-13, address >> 4): a constant add to the descriptor.
+    const uint64_t qdesc0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
+    const uint64_t qdesc1 = qdesc0 + (kSlotBytes >> 4);
+    const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
+    const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, 16384, 1024);
+    constexpr uint64_t kSlotDesc = kSlotBytes >> 4;
+    const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+    auto issue_s = [&](uint32_t tS, uint64_t qdesc, int slot) {
+      const uint64_t kdesc = dk0 + slot * kSlotDesc;
 #pragma unroll
-            for (int kk = 0; kk < C::kQKSteps; ++kk) {
-              const uint64_t off = kmajor_koff<kFp8>(kk) >> 4;
-              if (kFp8) mma_f8_ss(tS, qdesc + off, kdesc + off, C::kIdescQK, kk > 0);
-              else mma_f16_ss(tS, qdesc + off, kdesc + off, C::kIdescQK, kk > 0);
-            }
-            mma_commit(bar(kBarSFull + t));
-            mma_commit(bar(kBarKEmpty + slot));
-          } else {
-            mbar_arrive(bar(kBarKEmpty + slot));
-          }
+      for (int kk = 0; kk < C::kQKSteps; ++kk) {
+        const uint64_t off = kmajor_koff<kFp8>(kk) >> 4;
+        if (kFp8) mma_f8_ss(tS, qdesc + off, kdesc + off, C::kIdescQK, kk > 0);
+        else mma_f16_ss(tS, qdesc + off, kdesc + off, C::kIdescQK, kk > 0);
+      }
+    };
+    auto issue_pv = [&](uint32_t tO, uint32_t tS, int slot, bool started) {
+      const uint64_t vdesc = dv0 + slot * kSlotDesc;
+#pragma unroll
+      for (int kk = 0; kk < C::kPVSteps; ++kk) {
+        const uint32_t acc = (started || kk > 0) ? 1u : 0u;
+        const uint64_t bd = vdesc + ((kk * C::kKStep * 128) >> 4);
+        if (kFp8) mma_f8_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
+        else mma_f16_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
+      }
+    };
+    RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
+    int J, uses;
+    bool have = m.next(J, uses);
+    bool ok = true;
+    if (have) ok = __all_sync(kFull, mbar_wait(bar(kBarQ), 0, abort_flag));
+    uint32_t p_phase0 = 0, p_phase1 = 0;
+    bool o0_started = false, o1_started = false;
+    int pend = -1;  // union index of tile 1's entry whose P*V is not issued yet
+    int n = 0;
+    // O_1 += P_1 V for the pending entry, then release its V slot
+    auto flush_tile1 = [&]() -> bool {
+      const int ps = pend & 1;
+      const uint32_t pph = (pend >> 1) & 1;
+      if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag))) return false;
+      p_phase1 ^= 1;
+      if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), pph, abort_flag))) return false;
+      if (elect_one()) {
+        tc_fence_after();
+        issue_pv(tO1, tS1, ps, o1_started);
+        mma_commit(bar(kBarVEmpty + ps));
+      }
+      __syncwarp();
+      o1_started = true;
+      pend = -1;
+      return true;
+    };
+    while (ok && have) {
+      const int slot = n & 1;
+      const uint32_t ph = (n >> 1) & 1;
+      if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + slot), ph, abort_flag))) { ok = false; break; }
+      if (elect_one()) {
+        tc_fence_after();
+        if (uses & 1) {
+          issue_s(tS0, qdesc0, slot);
+          mma_commit(bar(kBarSFull + 0));
         }
-        if (mine) {
-          if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + t), p_phase, abort_flag))) { ok = false; break; }
-          p_phase ^= 1;
+      }
+      __syncwarp();
+      if (pend >= 0 && !flush_tile1()) { ok = false; break; }
+      if (elect_one()) {
+        if (uses & 2) {
+          issue_s(tS1, qdesc1, slot);
+          mma_commit(bar(kBarSFull + 1));
         }
+        mma_commit(bar(kBarKEmpty + slot));  // every S reading K_n has been issued
+      }
+      __syncwarp();
+      // The next union entry is read from the CSR arrays now, while the tensor pipe still holds
+      // this entry's MMAs and softmax 0 is running, not after O_0 += P_0 V (where the global-load
+      // latency would leave the pipe idle).
+      int uses_next;
+      const bool have_next = m.next(J, uses_next);
+      if (uses & 1) {
+        if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 0), p_phase0, abort_flag))) { ok = false; break; }
+        p_phase0 ^= 1;
         if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + slot), ph, abort_flag))) { ok = false; break; }
         if (elect_one()) {
-          if (mine) {
-            tc_fence_after();
-            const uint64_t vdesc = dv0 + slot * kSlotDesc;
-#pragma unroll
-            for (int kk = 0; kk < C::kPVSteps; ++kk) {
-              const uint32_t acc = (o_started || kk > 0) ? 1u : 0u;
-              const uint64_t bd = vdesc + ((kk * C::kKStep * 128) >> 4);
-              if (kFp8) mma_f8_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
-              else mma_f16_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
-            }
-            mma_commit(bar(kBarVEmpty + slot));
-          } else {
-            mbar_arrive(bar(kBarVEmpty + slot));
-          }
+          tc_fence_after();
+          issue_pv(tO0, tS0, slot, o0_started);
+          if (!(uses & 2)) mma_commit(bar(kBarVEmpty + slot));
         }
-        if (mine) o_started = true;
-        ++n;
+        __syncwarp();
+        o0_started = true;
       }
-      if (!ok) *abort_flag = 1;
-      if (elect_one()) {
-        mma_commit(bar(kBarODone + t));
-        // drain: every MMA issued by this warp completes before TMEM can be released
-        mma_commit(bar(kBarDrain + t));
-      }
-      volatile int never = 0;
-      mbar_wait(bar(kBarDrain + t), 0, &never);
+      if (uses & 2) pend = n;
+      ++n;
+      have = have_next;
+      uses = uses_next;
     }
+    if (ok && pend >= 0 && !flush_tile1()) ok = false;
+    if (!ok) *abort_flag = 1;
+    if (elect_one()) {
+      mma_commit(bar(kBarODone + 0));
+      mma_commit(bar(kBarODone + 1));
+      // drain: every MMA issued by this warp completes before TMEM can be released
+      mma_commit(bar(kBarDrain));
+    }
+    volatile int never = 0;
+    mbar_wait(bar(kBarDrain), 0, &never);
   }
   } else {
     setmaxnreg_inc<kSoftmaxRegs>();
@@ -450,16 +489,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool diag = (J == w.I);
         // the whole S row of this thread: 128 fp32 in registers (one TMEM read)
         uint32_t r[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, r + c * 32);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_wait_ld(r + c * 32);
+        tmem_ld32(tS, r);
+        tmem_ld32(tS + 32, r + 32);
+        tmem_wait_ld(r);
+        tmem_wait_ld(r + 32);
+        // second half in flight while the first half is masked and reduced
+        tmem_ld32(tS + 64, r + 64);
+        tmem_ld32(tS + 96, r + 96);
         if (diag) {  // token causal mask: key column > query row
 #pragma unroll
-          for (int j = 0; j < 128; ++j)
+          for (int j = 0; j < 64; ++j)
             if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
         }
-        const float mx = row_max128(r) * sl2;  // finite: key 0 is visible to every row
+        const float mx_lo = row_max64(r);
+        tmem_wait_ld(r + 64);
+        tmem_wait_ld(r + 96);
+        if (diag) {
+#pragma unroll
+          for (int j = 64; j < 128; ++j)
+            if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
+        }
+        const float mx = fmaxf(mx_lo, row_max64(r + 64)) * sl2;  // finite: key 0 is always visible
         // lazy rescale: move the reference max only when the block max exceeds it by > 2^8
         float corr = 1.f;
         if (mx > m_ref + kRescaleLog2) {
@@ -480,17 +530,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
         }
         // P = exp2(s * sl2 - m_ref), packed in place and written over S
-        const float rs = softmax_row_to_p<kFp8>(r, sl2, -m_ref);
-        if (kFp8) {
-          tmem_st32(tS, r);
-        } else {
-          tmem_st32(tS, r);
-          tmem_st32(tS + 32, r + 32);
-        }
+        // first half of P stored while the second half is computed
+        float rs = softmax_half_to_p<kFp8, 0>(r, sl2, -m_ref);
+        if (kFp8) tmem_st16(tS, r);
+        else tmem_st32(tS, r);
+        rs += softmax_half_to_p<kFp8, 64>(r, sl2, -m_ref);
+        if (kFp8) tmem_st16(tS + 16, r + 16);
+        else tmem_st32(tS + 32, r + 32);
         l_run += rs;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(kBarPReady + t));
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(bar(kBarPReady + t));
         ++it;
       }
       // epilogue: wait for the last P*V, normalise, store O (bf16) and the natural-log LSE
@@ -535,7 +586,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // ---- teardown: every role has drained its own async work ------------------------------
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
