@@ -20,7 +20,7 @@
 //
 // The tensor pipe buffers only a few MMA instructions, so the issuing thread must never stop for
 // long between groups.  One warp issues every MMA in a fixed order per union entry n:
-//     S_0(n) = Q_0 K_n^T | O_1 += P_1(n') V_n' | S_1(n) = Q_1 K_n^T | O_0 += P_0(n) V_n
+//     O_1 += P_1(n') V_n', S_1(n) = Q_1 K_n^T | O_0 += P_0(n) V_n, S_0(n + 1) = Q_0 K_{n+1}^T
 // where n' is tile 1's previous entry.  Softmax 0 of entry n then runs while the pipe executes
 // tile 1's P*V and S, and softmax 1 while it executes tile 0's P*V and next S, so the two
 // softmaxes alternate on the MUFU instead of contending for it.  S_t of an entry is always
@@ -99,21 +99,30 @@ __device__ __forceinline__ uint32_t kmajor_koff(int kk) {
 
 // Union of two CSR rows, consumed in list order.  Every entry of each row is visited exactly
 // once; entries outside [0, I] are skipped.  With ascending rows (as fpx_select writes them) the
-// union is ascending and shared blocks are visited once for both tiles.
+// union is ascending and shared blocks are visited once for both tiles.  The head of each row is
+// held in a register and its successor is loaded as soon as it is consumed, so the global-load
+// latency falls between two calls (one pipeline step) instead of inside one.
 struct RowMerge {
   const int32_t* ci;
   int a, a_end, b, b_end, I;
+  int va, vb;  // ci[a], ci[b] (INT_MAX past the end)
+  __device__ __forceinline__ RowMerge(const int32_t* ci_, int a_, int a_end_, int b_, int b_end_,
+                                      int I_)
+      : ci(ci_), a(a_), a_end(a_end_), b(b_), b_end(b_end_), I(I_) {
+    va = a < a_end ? ci[a] : INT_MAX;
+    vb = b < b_end ? ci[b] : INT_MAX;
+  }
   __device__ __forceinline__ bool ok(int J) const { return J >= 0 && J <= I; }
   __device__ __forceinline__ bool next(int& J, int& uses) {
-    while (a < a_end && !ok(ci[a])) ++a;
-    while (b < b_end && !ok(ci[b])) ++b;
+    while (a < a_end && !ok(va)) va = ++a < a_end ? ci[a] : INT_MAX;
+    while (b < b_end && !ok(vb)) vb = ++b < b_end ? ci[b] : INT_MAX;
     if (a >= a_end && b >= b_end) return false;
-    const int ja = a < a_end ? ci[a] : INT_MAX;
-    const int jb = b < b_end ? ci[b] : INT_MAX;
+    const int ja = a < a_end ? va : INT_MAX;
+    const int jb = b < b_end ? vb : INT_MAX;
     J = min(ja, jb);
     uses = (ja == J ? 1 : 0) | (jb == J ? 2 : 0);
-    if (ja == J) ++a;
-    if (jb == J) ++b;
+    if (ja == J) va = ++a < a_end ? ci[a] : INT_MAX;
+    if (jb == J) vb = ++b < b_end ? ci[b] : INT_MAX;
     return true;
   }
 };
@@ -163,13 +172,13 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
 #endif
 constexpr int kPolyEvery = FPX_POLY_EVERY;
 
-// Columns [J0, J0 + 64) of the S row in r become P, packed in place (bf16 pairs at r[J0 / 2 ..],
+// Columns [J0, J0 + N) of the S row in r become P, packed in place (bf16 pairs at r[J0 / 2 ..],
 // or e4m3 quads at r[J0 / 4 ..]); returns their sum.
-template <bool kFp8, int J0>
-__device__ __forceinline__ float softmax_half_to_p(uint32_t* r, float sl2, float neg_m) {
+template <bool kFp8, int J0, int N>
+__device__ __forceinline__ float softmax_part_to_p(uint32_t* r, float sl2, float neg_m) {
   float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int j = J0; j < J0 + 64; j += 2) {
+  for (int j = J0; j < J0 + N; j += 2) {
     float x0, x1, p0, p1;
     ffma2(x0, x1, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), sl2, sl2, neg_m, neg_m);
     constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
@@ -280,7 +289,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
+    RowMerge m(col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I);
     RowMerge peek = m;
     int J, uses;
     int n = 0;
@@ -371,7 +380,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         else mma_f16_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
       }
     };
-    RowMerge m{col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I};
+    RowMerge m(col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I);
     int J, uses;
     bool have = m.next(J, uses);
     bool ok = true;
@@ -380,37 +389,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     bool o0_started = false, o1_started = false;
     int pend = -1;  // union index of tile 1's entry whose P*V is not issued yet
     int n = 0;
-    // O_1 += P_1 V for the pending entry, then release its V slot
-    auto flush_tile1 = [&]() -> bool {
-      const int ps = pend & 1;
-      const uint32_t pph = (pend >> 1) & 1;
-      if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag))) return false;
-      p_phase1 ^= 1;
-      if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), pph, abort_flag))) return false;
-      if (elect_one()) {
-        tc_fence_after();
-        issue_pv(tO1, tS1, ps, o1_started);
-        mma_commit(bar(kBarVEmpty + ps));
+    // A P*V and the S that follows it in the same tile are issued back to back from one elected
+    // block: any wait or bookkeeping between them would leave the tensor pipe idle.
+    if (ok && have) {  // S_0 of the first entry
+      if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + 0), 0, abort_flag))) {
+        ok = false;
+      } else {
+        if (elect_one() && (uses & 1)) {
+          tc_fence_after();
+          issue_s(tS0, qdesc0, 0);
+          mma_commit(bar(kBarSFull + 0));
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      o1_started = true;
-      pend = -1;
-      return true;
-    };
+    }
     while (ok && have) {
       const int slot = n & 1;
       const uint32_t ph = (n >> 1) & 1;
-      if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + slot), ph, abort_flag))) { ok = false; break; }
+      // tile 1: O_1 += P_1 V of its previous entry, then S_1 of this entry
+      const bool pv1 = pend >= 0;
+      const int ps = pend & 1;
+      if (pv1) {
+        if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag))) { ok = false; break; }
+        p_phase1 ^= 1;
+        if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), (pend >> 1) & 1, abort_flag))) { ok = false; break; }
+      }
       if (elect_one()) {
         tc_fence_after();
-        if (uses & 1) {
-          issue_s(tS0, qdesc0, slot);
-          mma_commit(bar(kBarSFull + 0));
+        if (pv1) {
+          issue_pv(tO1, tS1, ps, o1_started);
+          mma_commit(bar(kBarVEmpty + ps));
         }
-      }
-      __syncwarp();
-      if (pend >= 0 && !flush_tile1()) { ok = false; break; }
-      if (elect_one()) {
         if (uses & 2) {
           issue_s(tS1, qdesc1, slot);
           mma_commit(bar(kBarSFull + 1));
@@ -418,29 +427,59 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(bar(kBarKEmpty + slot));  // every S reading K_n has been issued
       }
       __syncwarp();
-      // The next union entry is read from the CSR arrays now, while the tensor pipe still holds
-      // this entry's MMAs and softmax 0 is running, not after O_0 += P_0 V (where the global-load
-      // latency would leave the pipe idle).
-      int uses_next;
+      if (pv1) {
+        o1_started = true;
+        pend = -1;
+      }
+      // The next union entry (global loads of the CSR arrays) and its K tile, while this entry's
+      // MMAs run and softmax 0 works.
+      int uses_next = 0;
       const bool have_next = m.next(J, uses_next);
+      const int nslot = (n + 1) & 1;
+      if (have_next &&
+          !__all_sync(kFull, mbar_wait(bar(kBarKFull + nslot), ((n + 1) >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      const bool s0_next = have_next && (uses_next & 1);
+      // tile 0: O_0 += P_0 V of this entry, then S_0 of the next entry
       if (uses & 1) {
         if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 0), p_phase0, abort_flag))) { ok = false; break; }
         p_phase0 ^= 1;
         if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + slot), ph, abort_flag))) { ok = false; break; }
-        if (elect_one()) {
-          tc_fence_after();
+      }
+      if (elect_one()) {
+        tc_fence_after();
+        if (uses & 1) {
           issue_pv(tO0, tS0, slot, o0_started);
           if (!(uses & 2)) mma_commit(bar(kBarVEmpty + slot));
         }
-        __syncwarp();
-        o0_started = true;
+        if (s0_next) {
+          issue_s(tS0, qdesc0, nslot);
+          mma_commit(bar(kBarSFull + 0));
+        }
       }
+      __syncwarp();
+      if (uses & 1) o0_started = true;
       if (uses & 2) pend = n;
       ++n;
       have = have_next;
       uses = uses_next;
     }
-    if (ok && pend >= 0 && !flush_tile1()) ok = false;
+    if (ok && pend >= 0) {  // tile 1's last P*V
+      const int ps = pend & 1;
+      if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag)) ||
+          !__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), (pend >> 1) & 1, abort_flag))) {
+        ok = false;
+      } else {
+        if (elect_one()) {
+          tc_fence_after();
+          issue_pv(tO1, tS1, ps, o1_started);
+          mma_commit(bar(kBarVEmpty + ps));
+        }
+        __syncwarp();
+      }
+    }
     if (!ok) *abort_flag = 1;
     if (elect_one()) {
       mma_commit(bar(kBarODone + 0));
@@ -531,10 +570,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         // P = exp2(s * sl2 - m_ref), packed in place and written over S
         // first half of P stored while the second half is computed
-        float rs = softmax_half_to_p<kFp8, 0>(r, sl2, -m_ref);
+        float rs = softmax_part_to_p<kFp8, 0, 64>(r, sl2, -m_ref);
         if (kFp8) tmem_st16(tS, r);
         else tmem_st32(tS, r);
-        rs += softmax_half_to_p<kFp8, 64>(r, sl2, -m_ref);
+        rs += softmax_part_to_p<kFp8, 64, 64>(r, sl2, -m_ref);
         if (kFp8) tmem_st16(tS + 16, r + 16);
         else tmem_st32(tS + 32, r + 32);
         l_run += rs;
