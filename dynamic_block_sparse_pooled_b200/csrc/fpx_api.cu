@@ -185,7 +185,7 @@ fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, 
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   if (sz.nb == 0) return FPX_OK;
   if (launch_pool(d, p->dtype, q, k, qbar, kbar, t, s) != cudaSuccess) return FPX_ERR_CUDA;
-  if (launch_score(d, p->dtype, qbar, kbar, scores, t, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (launch_score(d, p->dtype, qbar, kbar, scores, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   return FPX_OK;
 }
 

@@ -13,8 +13,12 @@ cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cuda
 // fpx_block_scores: pool Q and K (fp32 means into qbar / kbar), then score pooled pairs.
 cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                         float* qbar, float* kbar, SeqTables t, cudaStream_t s);
+// Scores on the tensor cores (split-tf32, D = 128) when supported, else fp32 CUDA cores.
 cudaError_t launch_score(const ProblemDesc& p, fpx_dtype dt, const float* qbar, const float* kbar,
-                         float* scores, SeqTables t, cudaStream_t s);
+                         float* scores, SeqTables t, StatusBlock* st, cudaStream_t s);
+bool score_tc_supported(const ProblemDesc& p);
+cudaError_t launch_score_tc(const ProblemDesc& p, const float* qbar, const float* kbar,
+                            float* scores, SeqTables t, StatusBlock* st, cudaStream_t s);
 
 // fpx_select: row max + keep count, scan into row_ptr, emit col_idx.
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,

@@ -7,7 +7,8 @@
 //                   part of the search.
 //   * score_kernel  s_IJ = scale * <qbar_I, kbar_J> for the causal pairs J <= I, written as fp32
 //                   triangular rows.  64 x 64 register-tiled fp32 dot products out of shared
-//                   memory (the pooled vectors are L2-resident).
+//                   memory (the pooled vectors are L2-resident).  Used for D = 64; D = 128
+//                   takes the tensor-core kernel of fpx_score_sm100.cu.
 //   * select_*      per query-block row: row max, the alpha test exp(s - m) >= alpha OR sink OR
 //                   window, warp ballot/popc compaction into CSR (no sort, no cumulative sum
 //                   over scores).
@@ -312,8 +313,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ProblemDesc p,
 }
 
 cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, const float* kbar,
-                         float* scores, SeqTables t, cudaStream_t s) {
+                         float* scores, SeqTables t, StatusBlock* st, cudaStream_t s) {
   if (p.nb_total == 0) return cudaSuccess;
+  if (score_tc_supported(p)) return launch_score_tc(p, qbar, kbar, scores, t, st, s);
   const int nt = (p.nb_total + kScoreTile - 1) / kScoreTile;
   dim3 grid(nt * (nt + 1) / 2, p.hq);
   const size_t smem = 2 * sizeof(float) * p.d * kScoreTile;
