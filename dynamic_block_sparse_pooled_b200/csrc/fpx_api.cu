@@ -79,9 +79,9 @@ ProblemDesc make_desc(const fpx_problem* p, const Sizes& s) {
 size_t scratch_bytes(const fpx_problem* p, const Sizes& s, int which) {
   const size_t R = static_cast<size_t>(s.nb) * p->hq;
   switch (which) {
-    case 0:  // pooled Q and K, fp32
-      return align_up(sizeof(float) * s.nb * p->hq * p->d, 256) +
-             align_up(sizeof(float) * s.nb * p->hkv * p->d, 256);
+    case 0:  // pooled Q and K, fp32 (twice: tf32 hi and lo parts for the tensor-core scores)
+      return 2 * (align_up(sizeof(float) * s.nb * p->hq * p->d, 256) +
+                  align_up(sizeof(float) * s.nb * p->hkv * p->d, 256));
     case 1:  // row max, keep counts, per-CTA totals, overflow flag
       return align_up(sizeof(float) * R, 256) + align_up(sizeof(int32_t) * R, 256) +
              align_up(sizeof(int64_t) * (R / 8 + 1), 256) + 256;
@@ -180,12 +180,18 @@ fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, 
   StatusBlock* st = static_cast<StatusBlock*>(ws);
   const SeqTables t = seq_tables_at(ws, p->num_seqs);
   char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
+  const size_t qb = align_up(sizeof(float) * sz.nb * p->hq * p->d, 256);
+  const size_t kb = align_up(sizeof(float) * sz.nb * p->hkv * p->d, 256);
   float* qbar = reinterpret_cast<float*>(scratch);
-  float* kbar = reinterpret_cast<float*>(scratch + align_up(sizeof(float) * sz.nb * p->hq * p->d, 256));
+  float* kbar = reinterpret_cast<float*>(scratch + qb);
+  const bool tc = score_tc_supported(d);
+  float* qlo = tc ? reinterpret_cast<float*>(scratch + qb + kb) : nullptr;
+  float* klo = tc ? reinterpret_cast<float*>(scratch + 2 * qb + kb) : nullptr;
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   if (sz.nb == 0) return FPX_OK;
-  if (launch_pool(d, p->dtype, q, k, qbar, kbar, t, s) != cudaSuccess) return FPX_ERR_CUDA;
-  if (launch_score(d, p->dtype, qbar, kbar, scores, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (launch_pool(d, p->dtype, q, k, qbar, kbar, qlo, klo, t, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (launch_score(d, p->dtype, qbar, kbar, qlo, klo, scores, t, st, s) != cudaSuccess)
+    return FPX_ERR_CUDA;
   return FPX_OK;
 }
 

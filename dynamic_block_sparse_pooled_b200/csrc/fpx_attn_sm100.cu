@@ -632,6 +632,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 }
 
 // ---- host side ------------------------------------------------------------------------------
+}  // namespace sm100
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -646,21 +648,27 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [T, H, D] tensor -> 3-D map {D, H, T}, box {128 bytes, 1 head, 128 tokens}, 128B swizzle.
-static bool make_map(CUtensorMap* map, const void* base, int T, int H, int D, bool fp8) {
+bool make_tmap_rows128(CUtensorMap* map, const void* base, int T, int H, int D, int elem_bytes) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t es = fp8 ? 1 : 2;
+  const cuuint64_t es = static_cast<cuuint64_t>(elem_bytes);
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(T)};
   cuuint64_t strides[2] = {D * es, static_cast<cuuint64_t>(H) * D * es};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 1, 128};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult rc = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                   const_cast<void*>(base), dims, strides, box, estr,
+  const CUtensorMapDataType dt = elem_bytes == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult rc = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return rc == CUDA_SUCCESS;
+}
+
+namespace sm100 {
+static bool make_map(CUtensorMap* map, const void* base, int T, int H, int D, bool fp8) {
+  return make_tmap_rows128(map, base, T, H, D, fp8 ? 1 : 2);
 }
 
 }  // namespace sm100

@@ -1,6 +1,7 @@
 // fpx_internal.h -- host-side declarations shared by the fpx translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fpx_common.cuh"
@@ -11,14 +12,19 @@ namespace fpx {
 cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cudaStream_t s);
 
 // fpx_block_scores: pool Q and K (fp32 means into qbar / kbar), then score pooled pairs.
+// qlo / klo non-null: the means are stored split as tf32 hi (qbar / kbar) + lo (qlo / klo).
 cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
-                        float* qbar, float* kbar, SeqTables t, cudaStream_t s);
-// Scores on the tensor cores (split-tf32, D = 128) when supported, else fp32 CUDA cores.
+                        float* qbar, float* kbar, float* qlo, float* klo, SeqTables t,
+                        cudaStream_t s);
+// Scores on the tensor cores from the split means (qlo / klo non-null; requires
+// score_tc_supported), else fp32 CUDA cores from the plain means.
 cudaError_t launch_score(const ProblemDesc& p, fpx_dtype dt, const float* qbar, const float* kbar,
-                         float* scores, SeqTables t, StatusBlock* st, cudaStream_t s);
+                         const float* qlo, const float* klo, float* scores, SeqTables t,
+                         StatusBlock* st, cudaStream_t s);
 bool score_tc_supported(const ProblemDesc& p);
-cudaError_t launch_score_tc(const ProblemDesc& p, const float* qbar, const float* kbar,
-                            float* scores, SeqTables t, StatusBlock* st, cudaStream_t s);
+cudaError_t launch_score_tc(const ProblemDesc& p, const float* qhi, const float* khi,
+                            const float* qlo, const float* klo, float* scores, SeqTables t,
+                            StatusBlock* st, cudaStream_t s);
 
 // fpx_select: row max + keep count, scan into row_ptr, emit col_idx.
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
@@ -27,6 +33,10 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
                           int* overflow, SeqTables t, StatusBlock* st, cudaStream_t s);
 // CTAs of the select kernels (each owns 8 rows); the workspace holds one int64 per CTA.
 int select_ctas(const ProblemDesc& p);
+
+// [T, H, D] tensor -> 3-D TMA map {D, H, T} with box {128 bytes, 1, 128 rows} and 128B swizzle
+// (elem_bytes 1 = u8, 2 = bf16, 4 = fp32); false if the driver rejects it.
+bool make_tmap_rows128(CUtensorMap* map, const void* base, int T, int H, int D, int elem_bytes);
 
 // fpx_sparse_prefill: tile schedule, then one of the two attention kernels.
 // `units`: schedule the tensor-core kernel's two-head units instead of single CSR rows.

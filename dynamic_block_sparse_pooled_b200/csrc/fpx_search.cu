@@ -105,7 +105,10 @@ cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cuda
 
 // ------------------------------------------------------------------------------------------
 // pool: qbar[b, h, :] = mean of the valid rows of global block b.  grid.x = NB blocks,
-// grid.y = column chunks of Q's Hq*D row followed by those of K's Hkv*D row.
+// grid.y = column chunks of Q's Hq*D row followed by those of K's Hkv*D row.  With qlo / klo
+// given (tensor-core scores), the mean x is stored split for tf32 products: qbar = hi = x rounded
+// to tf32 (ties away from zero; the tensor core ignores the 13 low mantissa bits) and
+// qlo = lo = x - hi (exact), so that x = hi + lo.
 // ------------------------------------------------------------------------------------------
 constexpr int kPoolThreads = 128;
 
@@ -153,6 +156,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(ProblemDesc p, const
                                                             const T* __restrict__ k,
                                                             float* __restrict__ qbar,
                                                             float* __restrict__ kbar,
+                                                            float* __restrict__ qlo,
+                                                            float* __restrict__ klo,
                                                             const int32_t* __restrict__ blk_base,
                                                             const int32_t* __restrict__ valid,
                                                             int q_chunks) {
@@ -189,14 +194,32 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(ProblemDesc p, const
     Vec16<T>::add(__ldcs(reinterpret_cast<const int4*>(src + static_cast<int64_t>(r) * row_elems)),
                   acc);
   const float inv = 1.f / static_cast<float>(rows);
+  float* lo = is_q ? qlo : klo;
+  if (lo) {
+    lo += static_cast<int64_t>(b) * row_elems + c0;
+    float lv[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const float x = acc[i] * inv;
+      const float hi = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+      acc[i] = hi;
+      lv[i] = x - hi;
+    }
+#pragma unroll
+    for (int i = 0; i < V; i += 4)
+      *reinterpret_cast<float4*>(lo + i) = make_float4(lv[i], lv[i + 1], lv[i + 2], lv[i + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] *= inv;
+  }
 #pragma unroll
   for (int i = 0; i < V; i += 4)
-    *reinterpret_cast<float4*>(dst + i) =
-        make_float4(acc[i] * inv, acc[i + 1] * inv, acc[i + 2] * inv, acc[i + 3] * inv);
+    *reinterpret_cast<float4*>(dst + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
 }
 
 cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
-                        float* qbar, float* kbar, SeqTables t, cudaStream_t s) {
+                        float* qbar, float* kbar, float* qlo, float* klo, SeqTables t,
+                        cudaStream_t s) {
   const int32_t* blk_base = t.blk_base;
   if (p.nb_total == 0) return cudaSuccess;
   const int V = dt == FPX_F32 ? 4 : dt == FPX_BF16 ? 8 : 16;
@@ -208,17 +231,17 @@ cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const
     case FPX_F32:
       pool_kernel<float><<<grid, kPoolThreads, 0, s>>>(p, static_cast<const float*>(q),
                                                         static_cast<const float*>(k), qbar, kbar,
-                                                        blk_base, t.valid, q_chunks);
+                                                        qlo, klo, blk_base, t.valid, q_chunks);
       break;
     case FPX_BF16:
       pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, s>>>(
           p, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar,
-          kbar, blk_base, t.valid, q_chunks);
+          kbar, qlo, klo, blk_base, t.valid, q_chunks);
       break;
     default:
       pool_kernel<__nv_fp8_e4m3><<<grid, kPoolThreads, 0, s>>>(
           p, static_cast<const __nv_fp8_e4m3*>(q), static_cast<const __nv_fp8_e4m3*>(k), qbar,
-          kbar, blk_base, t.valid, q_chunks);
+          kbar, qlo, klo, blk_base, t.valid, q_chunks);
       break;
   }
   return cudaGetLastError();
@@ -313,9 +336,10 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ProblemDesc p,
 }
 
 cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, const float* kbar,
-                         float* scores, SeqTables t, StatusBlock* st, cudaStream_t s) {
+                         const float* qlo, const float* klo, float* scores, SeqTables t,
+                         StatusBlock* st, cudaStream_t s) {
   if (p.nb_total == 0) return cudaSuccess;
-  if (score_tc_supported(p)) return launch_score_tc(p, qbar, kbar, scores, t, st, s);
+  if (qlo && klo) return launch_score_tc(p, qbar, kbar, qlo, klo, scores, t, st, s);
   const int nt = (p.nb_total + kScoreTile - 1) / kScoreTile;
   dim3 grid(nt * (nt + 1) / 2, p.hq);
   const size_t smem = 2 * sizeof(float) * p.d * kScoreTile;
@@ -397,10 +421,19 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
     const float* row = scores + ri.base;
     const float m = row_max_warp(row, ri.len, lane);
     int cnt = 0;
-    for (int j0 = 0; j0 < ri.len; j0 += 32) {
-      const int j = j0 + lane;
-      const bool kp = j < ri.len && keep_block(row[j], m, alpha, j, ri.I, sink, window);
-      cnt += __popc(__ballot_sync(0xffffffffu, kp));
+    for (int j0 = 0; j0 < ri.len; j0 += 128) {  // four loads in flight per lane
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 32 * u + lane;
+        v[u] = j < ri.len ? row[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 32 * u + lane;
+        const bool kp = j < ri.len && keep_block(v[u], m, alpha, j, ri.I, sink, window);
+        cnt += __popc(__ballot_sync(0xffffffffu, kp));
+      }
     }
     if (lane == 0) {
       rowmax[r] = m;
@@ -508,12 +541,21 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
     const float* row = scores + ri.base;
     const float m = rowmax[r];
     int64_t out = base + s_off[rl];
-    for (int j0 = 0; j0 < ri.len; j0 += 32) {
-      const int j = j0 + lane;
-      const bool kp = j < ri.len && keep_block(__ldcs(row + j), m, alpha, j, ri.I, sink, window);
-      const unsigned bal = __ballot_sync(0xffffffffu, kp);
-      if (kp) col_idx[out + __popc(bal & ((1u << lane) - 1u))] = j;
-      out += __popc(bal);
+    for (int j0 = 0; j0 < ri.len; j0 += 128) {  // four loads in flight per lane
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 32 * u + lane;
+        v[u] = j < ri.len ? __ldcs(row + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 32 * u + lane;
+        const bool kp = j < ri.len && keep_block(v[u], m, alpha, j, ri.I, sink, window);
+        const unsigned bal = __ballot_sync(0xffffffffu, kp);
+        if (kp) col_idx[out + __popc(bal & ((1u << lane) - 1u))] = j;
+        out += __popc(bal);
+      }
     }
   }
 }
