@@ -3,6 +3,7 @@
 // fpx_query_status, which synchronises the stream it is given).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -14,8 +15,9 @@ using namespace fpx;
 namespace {
 
 struct Sizes {
-  int64_t nb = 0;   // NB
-  int64_t tri = 0;  // TRI
+  int64_t nb = 0;      // NB
+  int64_t tri = 0;     // TRI
+  int64_t nb_max = 0;  // blocks of the longest sequence
 };
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -39,6 +41,7 @@ fpx_status check_problem(const fpx_problem* p, Sizes* sz) {
     if (p->num_seqs != 1) return FPX_ERR_INVALID_ARG;
     s.nb = (static_cast<int64_t>(p->total_tokens) + p->block - 1) / p->block;
     s.tri = s.nb * (s.nb + 1) / 2;
+    s.nb_max = s.nb;
   } else {
     const int32_t* cu = p->cu_seqlens_h;
     if (cu[0] != 0 || cu[p->num_seqs] != p->total_tokens) return FPX_ERR_INVALID_ARG;
@@ -48,6 +51,7 @@ fpx_status check_problem(const fpx_problem* p, Sizes* sz) {
       const int64_t nb = (n + p->block - 1) / p->block;
       s.nb += nb;
       s.tri += nb * (nb + 1) / 2;
+      s.nb_max = std::max(s.nb_max, nb);
     }
   }
   // int32 CSR (row_ptr, col_idx) and int32 grid / row indices
@@ -76,15 +80,19 @@ ProblemDesc make_desc(const fpx_problem* p, const Sizes& s) {
   return d;
 }
 
+// Keep bitmask of the select stage: one 32-bit word per 32 key blocks of the longest row.
+int64_t mask_words(const Sizes& s) { return (s.nb_max + 31) / 32; }
+
 size_t scratch_bytes(const fpx_problem* p, const Sizes& s, int which) {
   const size_t R = static_cast<size_t>(s.nb) * p->hq;
   switch (which) {
     case 0:  // pooled Q and K, fp32 (twice: tf32 hi and lo parts for the tensor-core scores)
       return 2 * (align_up(sizeof(float) * s.nb * p->hq * p->d, 256) +
                   align_up(sizeof(float) * s.nb * p->hkv * p->d, 256));
-    case 1:  // row max, keep counts, per-CTA totals, overflow flag
+    case 1:  // row max, keep counts, per-CTA totals, overflow flag, keep bitmask
       return align_up(sizeof(float) * R, 256) + align_up(sizeof(int32_t) * R, 256) +
-             align_up(sizeof(int64_t) * (R / 8 + 1), 256) + 256;
+             align_up(sizeof(int64_t) * (R / 8 + 1), 256) + 256 +
+             align_up(sizeof(uint32_t) * R * mask_words(s), 256);
     case 2:  // tile schedule
       return align_up(sizeof(int32_t) * R, 256);
     default:
@@ -221,13 +229,15 @@ fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, in
                                                  align_up(sizeof(int32_t) * R, 256));
   int* overflow = reinterpret_cast<int*>(reinterpret_cast<char*>(cta_tot) +
                                          align_up(sizeof(int64_t) * (R / 8 + 1), 256));
+  uint32_t* mask = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(overflow) + 256);
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   // window / sink beyond any row are equivalent to "all": clamp so the device compare stays
   // in range
   const int sink = sink_blocks > d.nb_total ? d.nb_total + 1 : sink_blocks;
   const int window = window_blocks > d.nb_total ? d.nb_total + 1 : window_blocks;
   if (launch_select(d, scores, alpha, sink, window, row_ptr, col_idx, col_capacity, nnz_d, rowmax,
-                    counts, cta_tot, overflow, t, st, s) != cudaSuccess)
+                    counts, cta_tot, overflow, mask, static_cast<int>(mask_words(sz)), t, st,
+                    s) != cudaSuccess)
     return FPX_ERR_CUDA;
   return FPX_OK;
 }

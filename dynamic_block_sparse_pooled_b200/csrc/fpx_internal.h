@@ -26,11 +26,13 @@ cudaError_t launch_score_tc(const ProblemDesc& p, const float* qhi, const float*
                             const float* qlo, const float* klo, float* scores, SeqTables t,
                             StatusBlock* st, cudaStream_t s);
 
-// fpx_select: row max + keep count, scan into row_ptr, emit col_idx.
+// fpx_select: row max + keep count + keep bitmask (mask_words 32-bit words per row), scan into
+// row_ptr, emit col_idx from the bitmask.
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
                           int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
-                          int* overflow, SeqTables t, StatusBlock* st, cudaStream_t s);
+                          int* overflow, uint32_t* mask, int mask_words, SeqTables t,
+                          StatusBlock* st, cudaStream_t s);
 // CTAs of the select kernels (each owns 8 rows); the workspace holds one int64 per CTA.
 int select_ctas(const ProblemDesc& p);
 

@@ -357,9 +357,11 @@ cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, con
 
 // ------------------------------------------------------------------------------------------
 // select: a CTA owns 8 consecutive rows r = (h, s, I) (warp per row).
-//   count: row max, kept-block count per row, CTA total
+//   count: row max, kept-block count per row, CTA total, and the row's keep bitmask (bit J of
+//          word J / 32 at mask[r * mask_words + J / 32]: the ballot of the keep test)
 //   scan:  exclusive scan of the CTA totals (one CTA), nnz, capacity check
-//   emit:  per-CTA exclusive scan of its counts -> row_ptr; ballot/popc compaction -> col_idx
+//   emit:  per-CTA exclusive scan of its counts -> row_ptr; the bitmask (1/32 of the scores'
+//          bytes) compacted into col_idx with popc prefixes
 // ------------------------------------------------------------------------------------------
 constexpr int kSelWarps = 8;
 constexpr int kSelRowsPerWarp = 1;
@@ -408,7 +410,7 @@ __device__ __forceinline__ float row_max_warp(const float* __restrict__ row, int
 __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
     ProblemDesc p, const float* __restrict__ scores, float alpha, int sink, int window,
     float* __restrict__ rowmax, int32_t* __restrict__ counts, int64_t* __restrict__ cta_tot,
-    SeqTables t) {
+    uint32_t* __restrict__ mask, int mask_words, SeqTables t) {
   if (!*t.valid) return;
   __shared__ int w_tot[kSelWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -432,7 +434,10 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
       for (int u = 0; u < 4; ++u) {
         const int j = j0 + 32 * u + lane;
         const bool kp = j < ri.len && keep_block(v[u], m, alpha, j, ri.I, sink, window);
-        cnt += __popc(__ballot_sync(0xffffffffu, kp));
+        const unsigned bal = __ballot_sync(0xffffffffu, kp);
+        const int w = (j0 >> 5) + u;
+        if (lane == 0 && w < mask_words) mask[static_cast<int64_t>(r) * mask_words + w] = bal;
+        cnt += __popc(bal);
       }
     }
     if (lane == 0) {
@@ -508,10 +513,10 @@ __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
 }
 
 __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
-    ProblemDesc p, const float* __restrict__ scores, float alpha, int sink, int window,
-    const float* __restrict__ rowmax, const int32_t* __restrict__ counts,
-    const int64_t* __restrict__ cta_off, int32_t* __restrict__ row_ptr,
-    int32_t* __restrict__ col_idx, const int* __restrict__ overflow, SeqTables t) {
+    ProblemDesc p, const int32_t* __restrict__ counts, const int64_t* __restrict__ cta_off,
+    int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+    const int* __restrict__ overflow, const uint32_t* __restrict__ mask, int mask_words,
+    SeqTables t) {
   if (!*t.valid) return;
   __shared__ int32_t s_off[kSelRows];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -538,23 +543,17 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
     const int r = r0 + rl;
     if (r >= R) break;
     const RowInfo ri = row_info(p, t, r);
-    const float* row = scores + ri.base;
-    const float m = rowmax[r];
+    const uint32_t* words = mask + static_cast<int64_t>(r) * mask_words;
+    const int nw = (ri.len + 31) >> 5;
+    const unsigned below = (1u << lane) - 1u;
     int64_t out = base + s_off[rl];
-    for (int j0 = 0; j0 < ri.len; j0 += 128) {  // four loads in flight per lane
-      float v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j0 + 32 * u + lane;
-        v[u] = j < ri.len ? __ldcs(row + j) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j0 + 32 * u + lane;
-        const bool kp = j < ri.len && keep_block(v[u], m, alpha, j, ri.I, sink, window);
-        const unsigned bal = __ballot_sync(0xffffffffu, kp);
-        if (kp) col_idx[out + __popc(bal & ((1u << lane) - 1u))] = j;
-        out += __popc(bal);
+    for (int w0 = 0; w0 < nw; w0 += 32) {  // 32 words per load, one per lane
+      const uint32_t mine = w0 + lane < nw ? __ldcs(words + w0 + lane) : 0u;
+      const int n = min(32, nw - w0);
+      for (int q = 0; q < n; ++q) {
+        const uint32_t word = __shfl_sync(0xffffffffu, mine, q);
+        if ((word >> lane) & 1u) col_idx[out + __popc(word & below)] = 32 * (w0 + q) + lane;
+        out += __popc(word);
       }
     }
   }
@@ -565,12 +564,13 @@ int select_ctas(const ProblemDesc& p) { return (p.hq * p.nb_total + kSelRows - 1
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
                           int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
-                          int* overflow, SeqTables t, StatusBlock* st, cudaStream_t s) {
+                          int* overflow, uint32_t* mask, int mask_words, SeqTables t,
+                          StatusBlock* st, cudaStream_t s) {
   const int R = p.hq * p.nb_total;
   const int nblk = select_ctas(p);
   if (R > 0) {
     select_count_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
-                                                       counts, cta_tot, t);
+                                                       counts, cta_tot, mask, mask_words, t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -578,9 +578,8 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
                                                 overflow, t.valid, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || R == 0) return e;
-  select_emit_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
-                                                     counts, cta_tot, row_ptr, col_idx, overflow,
-                                                     t);
+  select_emit_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, counts, cta_tot, row_ptr, col_idx,
+                                                     overflow, mask, mask_words, t);
   return cudaGetLastError();
 }
 

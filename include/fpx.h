@@ -159,9 +159,10 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
  *   fpx_select_noalloc_max_bytes() bytes (2 MiB), which every GPU that loads the library holds
  *   until the process exits.  The caller still owns scores, row_ptr, col_idx and nnz_d.
  *   Same arguments and results as fpx_select, without ws / ws_bytes.
- *   Limits: the problem's fpx_workspace_bytes(p, 1) must not exceed the array (about 230,000
- *   query-block rows Hq * NB for a few sequences); larger problems return FPX_ERR_CAPACITY
- *   before anything is launched.  An invalid or unsupported problem returns FPX_ERR_INVALID_ARG.
+ *   Limits: the problem's fpx_workspace_bytes(p, 1) must not exceed the array (9 + 4 *
+ *   ceil(nb_max / 32) bytes per query-block row, nb_max = blocks of the longest sequence: about
+ *   160,000 rows Hq * NB when no sequence exceeds 32 blocks, about 28,000 at 512 blocks);
+ *   larger problems return FPX_ERR_CAPACITY before anything is launched.  An invalid or unsupported problem returns FPX_ERR_INVALID_ARG.
  *   Device-side conditions are visible through the outputs: nnz > col_capacity means nothing was
  *   written to col_idx; device cu_seqlens that disagree with the host mirror give an empty CSR.
  *   The first call on a device looks up the array's device address (once per device, with that
