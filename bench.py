@@ -38,6 +38,40 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 10  # plan+pool+score, plan+count+scan+emit, plan+order+attention
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch per workload,
+# from an ncu capture of the kernel built from sources whose digest is ATTN_TRAFFIC_DIGEST
+# (profiles/attn_tc_kernel_dram.md).  Reported as roofline.traffic only while the sources still
+# have that digest; any change to the kernel makes it null until it is measured again.
+ATTN_SOURCES = ("dynamic_block_sparse_pooled_b200/csrc/fpx_attn_sm100.cu",
+                "dynamic_block_sparse_pooled_b200/csrc/fpx_sm100.cuh",
+                "dynamic_block_sparse_pooled_b200/csrc/fpx_common.cuh")
+ATTN_TRAFFIC_DIGEST = "e550ae1ff7328781c6041853ccead8006436ae632ab50122e3382da086f1d222"
+ATTN_TRAFFIC = {
+    "llama8b_bf16_n131072": 3188644864 + 1083873024,
+    "llama8b_e4m3_n131072": 1201818112 + 1049840640,
+    "llama8b_bf16_n32768": 407646720 + 238250752,
+}
+
+
+def attn_sources_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attn_traffic(workload: str):
+    """Measured DRAM bytes of one attention launch, or None (not measured for this workload, or
+    the kernel sources changed since the capture)."""
+    if workload not in ATTN_TRAFFIC or ATTN_TRAFFIC_DIGEST is None:
+        return None
+    try:
+        return ATTN_TRAFFIC[workload] if attn_sources_digest() == ATTN_TRAFFIC_DIGEST else None
+    except OSError:
+        return None
+
 
 def peaks():
     try:
@@ -260,7 +294,8 @@ def run_ours(args, rank, world, device):
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(achieved, 2),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
                      "peak_kind": f"{pk_kind} bf16 sustained" + (" x2 (fp8)" if w.dtype == "e4m3" else ""),
-                     "traffic": None,
+                     "traffic": attn_traffic(w.name),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "per_launch": "executed FLOP = 4*B^2*D*nnz (every kept 128x128 tile)"},
         "e2e": {"value": round(aggregate_value(flops, world, e2e_ms), 3),
                 "unit": "TFLOP/s (dense-equivalent, host buffers, copies included)",
