@@ -170,6 +170,41 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------------------------
 
+def sdpa_baseline(w, dev, cu, device, reps=2):
+    """Library baseline on the same inputs: PyTorch SDPA causal attention (dense, i.e. every
+    causal tile; K/V expanded to the Q heads), restricted to the fused flash / cuDNN backends so
+    that it can never fall back to the O(N^2)-memory math path.  bf16 workloads only."""
+    if w.dtype != "bf16":
+        return {"unavailable": "SDPA takes no e4m3 / fp32-parity configuration here"}
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        F = torch.nn.functional
+        g = w.hq // w.hkv
+        seqs = [(int(cu[i]), int(cu[i + 1])) for i in range(len(cu) - 1) if cu[i + 1] > cu[i]]
+
+        def run():
+            for a, b in seqs:
+                qq = dev["q"][a:b].transpose(0, 1).unsqueeze(0)
+                kk = dev["k"][a:b].repeat_interleave(g, dim=1).transpose(0, 1).unsqueeze(0)
+                vv = dev["v"][a:b].repeat_interleave(g, dim=1).transpose(0, 1).unsqueeze(0)
+                F.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+
+        with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.CUDNN_ATTENTION]):
+            run()
+            torch.cuda.synchronize(device)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                run()
+            b.record()
+            torch.cuda.synchronize(device)
+        ms = a.elapsed_time(b) / reps
+        return {"ms": round(ms, 3), "dense_equiv_tflops": round(dense_flops(w) / (ms * 1e-3) / 1e12, 1),
+                "what": "torch SDPA is_causal (flash/cuDNN backends), K/V head expansion included"}
+    except Exception as e:  # a missing backend is reported, never a fallback
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
+
+
 def run_ours(args, rank, world, device):
     import dynamic_block_sparse_pooled_b200 as fpx
 
@@ -302,6 +337,7 @@ def run_ours(args, rank, world, device):
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "sdpa_baseline": sdpa_baseline(w, dev, cu, device) if not args.no_sdpa else None,
         "clocks": clk.summary(),
     }
     return res, w, data
@@ -391,6 +427,7 @@ def main():
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sdpa", action="store_true", help="skip the PyTorch SDPA baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
