@@ -75,3 +75,13 @@ def test_reference_arm_rank_contract():
     assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_traffic_is_reported_only_for_the_measured_sources(monkeypatch):
+    # sources with the recorded digest: the measured bytes; a workload never measured: null
+    monkeypatch.setattr(bench, "ATTN_TRAFFIC_DIGEST", bench.attn_sources_digest())
+    assert bench.attn_traffic("llama8b_bf16_n131072") == bench.ATTN_TRAFFIC["llama8b_bf16_n131072"]
+    assert bench.attn_traffic("varlen8_bf16_t264192") is None
+    # kernel sources that differ from the captured ones: null
+    monkeypatch.setattr(bench, "ATTN_TRAFFIC_DIGEST", "0" * 64)
+    assert bench.attn_traffic("llama8b_bf16_n131072") is None
