@@ -30,7 +30,8 @@ STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "misaligned po
 EXPORTS = ("fpx_num_blocks", "fpx_scores_elems", "fpx_rows", "fpx_max_nnz", "fpx_workspace_bytes",
            "fpx_clear_status", "fpx_query_status", "fpx_status_string", "fpx_block_scores",
            "fpx_select", "fpx_sparse_prefill", "fpx_attention_path", "fpx_select_noalloc",
-           "fpx_select_noalloc_max_bytes", "fpx_diag_bounded_wait")
+           "fpx_select_noalloc_max_bytes", "fpx_diag_bounded_wait", "fpx_block_scores_paged",
+           "fpx_sparse_prefill_paged")
 
 
 class FpxError(RuntimeError):
@@ -47,6 +48,21 @@ class Problem(ctypes.Structure):
                 ("block", ctypes.c_int32), ("dtype", ctypes.c_int),
                 ("q_scale_d", ctypes.c_void_p), ("k_scale_d", ctypes.c_void_p),
                 ("v_scale_d", ctypes.c_void_p), ("softmax_scale", ctypes.c_float)]
+
+
+class PagedKV(ctypes.Structure):
+    """Mirror of ``fpx_paged_kv``."""
+    _fields_ = [("block_table_d", ctypes.c_void_p), ("pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
+
+
+def paged_kv(block_table: torch.Tensor, num_pages: int) -> PagedKV:
+    """Describes a page table: device int32 [num_seqs, pages_per_seq] of page indices."""
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 [num_seqs, pages_per_seq] tensor")
+    kv = PagedKV(block_table.data_ptr(), block_table.shape[1], int(num_pages))
+    kv._keep = block_table  # the table must outlive the calls that use it
+    return kv
 
 
 _lib = None
@@ -89,6 +105,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fpx_select_noalloc_max_bytes.restype = sz
     lib.fpx_diag_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
     lib.fpx_diag_bounded_wait.restype = ctypes.c_int
+    K = ctypes.POINTER(PagedKV)
+    lib.fpx_block_scores_paged.argtypes = [P, vp, vp, K, vp, vp, sz, vp]
+    lib.fpx_block_scores_paged.restype = ctypes.c_int
+    lib.fpx_sparse_prefill_paged.argtypes = [P, vp, vp, vp, K, vp, vp, vp, vp, vp, sz, vp]
+    lib.fpx_sparse_prefill_paged.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -238,6 +259,35 @@ def sparse_prefill(pf: Prefill, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
     check(load().fpx_sparse_prefill(pf.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                     _ptr(col_idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
                                     _stream(stream)), "fpx_sparse_prefill")
+    return o, lse
+
+
+def block_scores_paged(pf: Prefill, q: torch.Tensor, k_cache: torch.Tensor, kv: PagedKV,
+                       ws: torch.Tensor, scores: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """fpx_block_scores_paged: K from the paged cache [num_pages, block, Hkv, D]."""
+    if scores is None:
+        scores = torch.empty(pf.struct.hq * pf.tri, dtype=torch.float32, device=q.device)
+    check(load().fpx_block_scores_paged(pf.ptr, _ptr(q), _ptr(k_cache), ctypes.byref(kv),
+                                        _ptr(scores), _ptr(ws), ws.numel(), _stream(stream)),
+          "fpx_block_scores_paged")
+    return scores
+
+
+def sparse_prefill_paged(pf: Prefill, q: torch.Tensor, k_cache: torch.Tensor,
+                         v_cache: torch.Tensor, kv: PagedKV, row_ptr: torch.Tensor,
+                         col_idx: torch.Tensor, ws: torch.Tensor,
+                         o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         stream=None):
+    """fpx_sparse_prefill_paged: K and V from the paged caches -> (O, LSE)."""
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    check(load().fpx_sparse_prefill_paged(pf.ptr, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          ctypes.byref(kv), _ptr(row_ptr), _ptr(col_idx),
+                                          _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "fpx_sparse_prefill_paged")
     return o, lse
 
 

@@ -77,7 +77,26 @@ ProblemDesc make_desc(const fpx_problem* p, const Sizes& s) {
   d.q_scale = fp8 ? p->q_scale_d : nullptr;
   d.k_scale = fp8 ? p->k_scale_d : nullptr;
   d.v_scale = fp8 ? p->v_scale_d : nullptr;
+  d.page_table = nullptr;
+  d.pages_per_seq = 0;
+  d.num_pages = 0;
   return d;
+}
+
+// Host checks of a paged K / V description against the problem; fills the descriptor fields.
+fpx_status apply_paged(const fpx_problem* p, const Sizes& s, const fpx_paged_kv* kv,
+                       ProblemDesc* d) {
+  if (!kv || !kv->block_table_d) return FPX_ERR_INVALID_ARG;
+  if (kv->num_pages < 1 || kv->pages_per_seq < s.nb_max || kv->pages_per_seq < 1)
+    return FPX_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(kv->num_pages) * p->block > INT32_MAX ||
+      static_cast<int64_t>(kv->pages_per_seq) * p->num_seqs > INT32_MAX)
+    return FPX_ERR_UNSUPPORTED;
+  if (!aligned(kv->block_table_d, 4)) return FPX_ERR_ALIGNMENT;
+  d->page_table = kv->block_table_d;
+  d->pages_per_seq = kv->pages_per_seq;
+  d->num_pages = kv->num_pages;
+  return FPX_OK;
 }
 
 // Keep bitmask of the select stage: one 32-bit word per 32 key blocks of the longest row.
@@ -175,8 +194,9 @@ int fpx_attention_path(const fpx_problem* p) {
   return attn_tc_supported(make_desc(p, s), p->dtype) ? 1 : 0;
 }
 
-fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, float* scores,
-                            void* ws, size_t ws_bytes, fpx_stream_t stream) {
+static fpx_status block_scores_impl(const fpx_problem* p, const void* q, const void* k,
+                                    const fpx_paged_kv* kv, float* scores, void* ws,
+                                    size_t ws_bytes, fpx_stream_t stream) {
   Sizes sz;
   fpx_status rc = check_problem(p, &sz);
   if (rc != FPX_OK) return rc;
@@ -184,7 +204,8 @@ fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, 
   if (p->total_tokens > 0 && (!q || !k || !scores)) return FPX_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(scores, 4)) return FPX_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const ProblemDesc d = make_desc(p, sz);
+  ProblemDesc d = make_desc(p, sz);
+  if (kv && (rc = apply_paged(p, sz, kv, &d)) != FPX_OK) return rc;
   StatusBlock* st = static_cast<StatusBlock*>(ws);
   const SeqTables t = seq_tables_at(ws, p->num_seqs);
   char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
@@ -197,10 +218,23 @@ fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, 
   float* klo = tc ? reinterpret_cast<float*>(scratch + 2 * qb + kb) : nullptr;
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   if (sz.nb == 0) return FPX_OK;
-  if (launch_pool(d, p->dtype, q, k, qbar, kbar, qlo, klo, t, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (launch_pool(d, p->dtype, q, k, qbar, kbar, qlo, klo, t, st, s) != cudaSuccess)
+    return FPX_ERR_CUDA;
   if (launch_score(d, p->dtype, qbar, kbar, qlo, klo, scores, t, st, s) != cudaSuccess)
     return FPX_ERR_CUDA;
   return FPX_OK;
+}
+
+fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, float* scores,
+                            void* ws, size_t ws_bytes, fpx_stream_t stream) {
+  return block_scores_impl(p, q, k, nullptr, scores, ws, ws_bytes, stream);
+}
+
+fpx_status fpx_block_scores_paged(const fpx_problem* p, const void* q, const void* k_cache,
+                                  const fpx_paged_kv* kv, float* scores, void* ws,
+                                  size_t ws_bytes, fpx_stream_t stream) {
+  if (!kv) return FPX_ERR_INVALID_ARG;
+  return block_scores_impl(p, q, k_cache, kv, scores, ws, ws_bytes, stream);
 }
 
 fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, int32_t sink_blocks,
@@ -242,9 +276,11 @@ fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, in
   return FPX_OK;
 }
 
-fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k, const void* v,
-                              const int32_t* row_ptr, const int32_t* col_idx, void* o,
-                              float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream) {
+static fpx_status sparse_prefill_impl(const fpx_problem* p, const void* q, const void* k,
+                                      const void* v, const fpx_paged_kv* kv,
+                                      const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                                      float* lse, void* ws, size_t ws_bytes,
+                                      fpx_stream_t stream) {
   Sizes sz;
   fpx_status rc = check_problem(p, &sz);
   if (rc != FPX_OK) return rc;
@@ -254,7 +290,11 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
       !aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
     return FPX_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const ProblemDesc d = make_desc(p, sz);
+  ProblemDesc d = make_desc(p, sz);
+  if (kv) {
+    if ((rc = apply_paged(p, sz, kv, &d)) != FPX_OK) return rc;
+    if (!attn_tc_supported(d, p->dtype)) return FPX_ERR_UNSUPPORTED;  // paged: tensor-core path
+  }
   StatusBlock* st = static_cast<StatusBlock*>(ws);
   const SeqTables t = seq_tables_at(ws, p->num_seqs);
   char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
@@ -273,6 +313,21 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
   return launch_attn_simt(d, p->dtype, q, k, v, row_ptr, col_idx, o, lse, t, order, st, s) == cudaSuccess
              ? FPX_OK
              : FPX_ERR_CUDA;
+}
+
+fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k, const void* v,
+                              const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                              float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream) {
+  return sparse_prefill_impl(p, q, k, v, nullptr, row_ptr, col_idx, o, lse, ws, ws_bytes, stream);
+}
+
+fpx_status fpx_sparse_prefill_paged(const fpx_problem* p, const void* q, const void* k_cache,
+                                    const void* v_cache, const fpx_paged_kv* kv,
+                                    const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                                    float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream) {
+  if (!kv) return FPX_ERR_INVALID_ARG;
+  return sparse_prefill_impl(p, q, k_cache, v_cache, kv, row_ptr, col_idx, o, lse, ws, ws_bytes,
+                             stream);
 }
 
 }  // extern "C"

@@ -311,7 +311,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     while (m.next(J, uses)) {
       const int slot = n & 1;
       const uint32_t ph = (n >> 1) & 1;
-      const int kv_tok = w.tok0 + J * kTileN;
+      // first K / V row of block J (its page when K / V are paged); a page index outside the
+      // cache is recorded and read past the end of the map (TMA fills zeros there)
+      int64_t kv_row = kv_block_row(p, w.s, J, w.tok0);
+      if (kv_row < 0) {
+        if (elect_one()) record_error(st, FPX_ERR_DEVICE_INPUT, 34, w.s, J);
+        kv_row = static_cast<int64_t>(p.num_pages) * kTileN;
+      }
+      const int kv_tok = static_cast<int>(kv_row);
       if (!__all_sync(kFull, mbar_wait(bar(kBarKEmpty + slot), ph ^ 1, abort_flag))) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(bar(kBarKFull + slot), C::kTileBytes);
@@ -691,9 +698,10 @@ cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, co
   if (units == 0) return cudaSuccess;
   const bool fp8 = dt == FPX_E4M3;
   CUtensorMap mq, mk, mv;
+  const int kv_rows = p.page_table ? p.num_pages * p.block : p.total_tokens;
   if (!make_map(&mq, q, p.total_tokens, p.hq, p.d, fp8) ||
-      !make_map(&mk, k, p.total_tokens, p.hkv, p.d, fp8) ||
-      !make_map(&mv, v, p.total_tokens, p.hkv, p.d, fp8)) {
+      !make_map(&mk, k, kv_rows, p.hkv, p.d, fp8) ||
+      !make_map(&mv, v, kv_rows, p.hkv, p.d, fp8)) {
     *encode_failed = true;
     return cudaErrorInvalidValue;
   }

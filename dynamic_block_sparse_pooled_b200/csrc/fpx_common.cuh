@@ -63,7 +63,20 @@ struct ProblemDesc {
   const float* q_scale;
   const float* k_scale;
   const float* v_scale;
+  // paged K / V (nullptr => K and V are packed like Q): K / V row of token t of key block J of
+  // sequence s = page_table[s * pages_per_seq + J] * block + t, pages of `block` tokens
+  const int32_t* page_table;
+  int32_t pages_per_seq;
+  int32_t num_pages;
 };
+
+// First K / V row of key block J of sequence s (tok0 = the sequence's first token), or -1 when a
+// paged table names a page outside [0, num_pages).
+__device__ __forceinline__ int64_t kv_block_row(const ProblemDesc& p, int s, int J, int tok0) {
+  if (!p.page_table) return static_cast<int64_t>(tok0) + static_cast<int64_t>(J) * p.block;
+  const int pg = p.page_table[static_cast<int64_t>(s) * p.pages_per_seq + J];
+  return (pg < 0 || pg >= p.num_pages) ? -1 : static_cast<int64_t>(pg) * p.block;
+}
 
 __device__ __forceinline__ void record_error(StatusBlock* st, int code, int where, int d0 = 0,
                                              int d1 = 0) {

@@ -15,7 +15,7 @@ cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cuda
 // qlo / klo non-null: the means are stored split as tf32 hi (qbar / kbar) + lo (qlo / klo).
 cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                         float* qbar, float* kbar, float* qlo, float* klo, SeqTables t,
-                        cudaStream_t s);
+                        StatusBlock* st, cudaStream_t s);
 // Scores on the tensor cores from the split means (qlo / klo non-null; requires
 // score_tc_supported), else fp32 CUDA cores from the plain means.
 cudaError_t launch_score(const ProblemDesc& p, fpx_dtype dt, const float* qbar, const float* kbar,

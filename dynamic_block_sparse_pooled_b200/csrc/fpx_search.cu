@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(ProblemDesc p, const
                                                             float* __restrict__ klo,
                                                             const int32_t* __restrict__ blk_base,
                                                             const int32_t* __restrict__ valid,
-                                                            int q_chunks) {
+                                                            int q_chunks, StatusBlock* st) {
   constexpr int V = Vec16<T>::N;
   if (!*valid) return;
   const int b = blockIdx.x;
@@ -175,7 +175,23 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(ProblemDesc p, const
   const int row_elems = (is_q ? p.hq : p.hkv) * p.d;
   const int c0 = (chunk * kPoolThreads + threadIdx.x) * V;
   if (c0 >= row_elems) return;
-  const T* src = (is_q ? q : k) + tok0 * row_elems + c0;
+  // K rows come from the block's page when K is paged
+  const int64_t row0 = is_q ? tok0 : kv_block_row(p, s, I, seq_start(p, s));
+  if (row0 < 0) {  // page index outside the cache: recorded, the block's mean is zero
+    if (threadIdx.x == 0) record_error(st, FPX_ERR_DEVICE_INPUT, 4, s, I);
+    float* dst = kbar + static_cast<int64_t>(b) * row_elems + c0;
+#pragma unroll
+    for (int i = 0; i < V; i += 4)
+      *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (klo) {
+      float* lo = klo + static_cast<int64_t>(b) * row_elems + c0;
+#pragma unroll
+      for (int i = 0; i < V; i += 4)
+        *reinterpret_cast<float4*>(lo + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
+  const T* src = (is_q ? q : k) + row0 * row_elems + c0;
   float* dst = (is_q ? qbar : kbar) + static_cast<int64_t>(b) * row_elems + c0;
 
   float acc[V];
@@ -219,7 +235,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(ProblemDesc p, const
 
 cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                         float* qbar, float* kbar, float* qlo, float* klo, SeqTables t,
-                        cudaStream_t s) {
+                        StatusBlock* st, cudaStream_t s) {
   const int32_t* blk_base = t.blk_base;
   if (p.nb_total == 0) return cudaSuccess;
   const int V = dt == FPX_F32 ? 4 : dt == FPX_BF16 ? 8 : 16;
@@ -231,17 +247,17 @@ cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const
     case FPX_F32:
       pool_kernel<float><<<grid, kPoolThreads, 0, s>>>(p, static_cast<const float*>(q),
                                                         static_cast<const float*>(k), qbar, kbar,
-                                                        qlo, klo, blk_base, t.valid, q_chunks);
+                                                        qlo, klo, blk_base, t.valid, q_chunks, st);
       break;
     case FPX_BF16:
       pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, s>>>(
           p, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar,
-          kbar, qlo, klo, blk_base, t.valid, q_chunks);
+          kbar, qlo, klo, blk_base, t.valid, q_chunks, st);
       break;
     default:
       pool_kernel<__nv_fp8_e4m3><<<grid, kPoolThreads, 0, s>>>(
           p, static_cast<const __nv_fp8_e4m3*>(q), static_cast<const __nv_fp8_e4m3*>(k), qbar,
-          kbar, qlo, klo, blk_base, t.valid, q_chunks);
+          kbar, qlo, klo, blk_base, t.valid, q_chunks, st);
       break;
   }
   return cudaGetLastError();

@@ -151,6 +151,37 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
                               float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream);
 
 /*
+ * Paged K / V (FlashPrefill V2 abstract: native paged KV cache and continuous batching, as
+ * inference servers keep the cache).  K and V live in a cache of fixed-size pages of `block`
+ * tokens, [num_pages, block, hkv, d] in the problem's dtype (the same element layout as a
+ * packed [num_pages * block, hkv, d] tensor, 16-byte aligned); Q stays packed by cu_seqlens.
+ *   block_table_d  device int32 [num_seqs, pages_per_seq]: entry (s, J) is the page holding key
+ *                  block J of sequence s (tokens J * block .. of that sequence); entries with
+ *                  J >= nb_s are never read.  pages_per_seq >= the longest sequence's nb_s.
+ *   num_pages      pages in the cache (num_pages * block <= INT32_MAX).
+ * Rows of a sequence's last page beyond its length must hold finite values (they are multiplied
+ * by zero).  A page index outside [0, num_pages) is recorded as FPX_ERR_DEVICE_INPUT and read as
+ * zeros.  Same results as the packed entry points on the same data, bit for bit.
+ */
+typedef struct {
+  const int32_t* block_table_d;
+  int32_t pages_per_seq;
+  int32_t num_pages;
+} fpx_paged_kv;
+
+/* fpx_block_scores with K read from the paged cache (any dtype / d / block). */
+fpx_status fpx_block_scores_paged(const fpx_problem* p, const void* q, const void* k_cache,
+                                  const fpx_paged_kv* kv, float* scores, void* ws,
+                                  size_t ws_bytes, fpx_stream_t stream);
+
+/* fpx_sparse_prefill with K and V read from the paged caches.  Tensor-core path only (bf16 or
+ * e4m3, d = 128, block = 128; fpx_attention_path(p) == 1), else FPX_ERR_UNSUPPORTED. */
+fpx_status fpx_sparse_prefill_paged(const fpx_problem* p, const void* q, const void* k_cache,
+                                    const void* v_cache, const fpx_paged_kv* kv,
+                                    const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                                    float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream);
+
+/*
  * Allocation-free variant of fpx_select (the paper has no counterpart; it exists for callers).
  *   Some callers cannot allocate device memory where they run: a plugin whose host framework
  *   owns all device memory and offers no scratch buffer, or latency-critical code that must not

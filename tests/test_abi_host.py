@@ -128,3 +128,29 @@ def test_status_strings():
     lib = fpx.load()
     for code in range(-7, 1):
         assert lib.fpx_status_string(code)
+
+
+def test_paged_argument_errors():
+    lib = fpx.load()
+    p, keep = make([300, 1000])  # nb_s = 3 and 8
+    ref = ctypes.byref(p)
+    big = 1 << 30
+    a = 0x100000
+    ok_kv = fpx.PagedKV(0x3000, 8, 64)
+    assert lib.fpx_block_scores_paged(ref, a, a, None, a, a, big, None) == -1          # no table
+    assert lib.fpx_block_scores_paged(ref, a, a, ctypes.byref(fpx.PagedKV(None, 8, 64)), a, a,
+                                      big, None) == -1
+    assert lib.fpx_block_scores_paged(ref, a, a, ctypes.byref(fpx.PagedKV(0x3000, 7, 64)), a, a,
+                                      big, None) == -1                                  # < nb_max
+    assert lib.fpx_block_scores_paged(ref, a, a, ctypes.byref(fpx.PagedKV(0x3000, 8, 0)), a, a,
+                                      big, None) == -1                                  # no pages
+    assert lib.fpx_block_scores_paged(ref, a, a, ctypes.byref(fpx.PagedKV(0x3002, 8, 64)), a, a,
+                                      big, None) == -3                                  # misaligned
+    assert lib.fpx_sparse_prefill_paged(ref, a, a, a, None, a, a, a, a, a, big, None) == -1
+    # paged attention runs on the tensor-core path only
+    pf, keep2 = make([300, 1000], dtype=fpx.F32)
+    assert lib.fpx_sparse_prefill_paged(ctypes.byref(pf), a, a, a, ctypes.byref(ok_kv), a, a, a,
+                                        a, a, big, None) == -2
+    pd, keep3 = make([300, 1000], d=64)
+    assert lib.fpx_sparse_prefill_paged(ctypes.byref(pd), a, a, a, ctypes.byref(ok_kv), a, a, a,
+                                        a, a, big, None) == -2
