@@ -31,7 +31,7 @@ EXPORTS = ("fpx_num_blocks", "fpx_scores_elems", "fpx_rows", "fpx_max_nnz", "fpx
            "fpx_clear_status", "fpx_query_status", "fpx_status_string", "fpx_block_scores",
            "fpx_select", "fpx_sparse_prefill", "fpx_attention_path", "fpx_select_noalloc",
            "fpx_select_noalloc_max_bytes", "fpx_diag_bounded_wait", "fpx_block_scores_paged",
-           "fpx_sparse_prefill_paged")
+           "fpx_sparse_prefill_paged", "fpx_block_scores_rescue", "fpx_select_rescue")
 
 
 class FpxError(RuntimeError):
@@ -110,6 +110,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fpx_block_scores_paged.restype = ctypes.c_int
     lib.fpx_sparse_prefill_paged.argtypes = [P, vp, vp, vp, K, vp, vp, vp, vp, vp, sz, vp]
     lib.fpx_sparse_prefill_paged.restype = ctypes.c_int
+    lib.fpx_block_scores_rescue.argtypes = [P, vp, vp, K, vp, vp, vp, vp, sz, vp]
+    lib.fpx_block_scores_rescue.restype = ctypes.c_int
+    lib.fpx_select_rescue.argtypes = [P, vp, vp, vp, f32, f32, i32, i32, vp, vp, i64, vp, vp, sz,
+                                      vp]
+    lib.fpx_select_rescue.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -289,6 +294,36 @@ def sparse_prefill_paged(pf: Prefill, q: torch.Tensor, k_cache: torch.Tensor,
                                           _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
                                           _stream(stream)), "fpx_sparse_prefill_paged")
     return o, lse
+
+
+def block_scores_rescue(pf: Prefill, q: torch.Tensor, k: torch.Tensor, ws: torch.Tensor,
+                        kv: Optional[PagedKV] = None, stream=None):
+    """fpx_block_scores_rescue -> (scores [Hq * TRI], qnorm [Hq, NB], radius [Hkv, NB])."""
+    nb = pf.rows // pf.struct.hq
+    scores = torch.empty(pf.struct.hq * pf.tri, dtype=torch.float32, device=q.device)
+    qnorm = torch.empty((pf.struct.hq, nb), dtype=torch.float32, device=q.device)
+    radius = torch.empty((pf.struct.hkv, nb), dtype=torch.float32, device=q.device)
+    check(load().fpx_block_scores_rescue(pf.ptr, _ptr(q), _ptr(k),
+                                         ctypes.byref(kv) if kv is not None else None,
+                                         _ptr(scores), _ptr(qnorm), _ptr(radius), _ptr(ws),
+                                         ws.numel(), _stream(stream)), "fpx_block_scores_rescue")
+    return scores, qnorm, radius
+
+
+def select_rescue(pf: Prefill, scores: torch.Tensor, qnorm: torch.Tensor, radius: torch.Tensor,
+                  alpha: float, alpha_rescue: float, ws: torch.Tensor, sink_blocks: int = 1,
+                  window_blocks: int = 1, stream=None):
+    """fpx_select_rescue -> (row_ptr, col_idx, nnz) of the base OR rescue selection."""
+    dev = scores.device
+    row_ptr = torch.empty(pf.rows + 1, dtype=torch.int32, device=dev)
+    cap = pf.struct.hq * pf.tri
+    col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    check(load().fpx_select_rescue(pf.ptr, _ptr(scores), _ptr(qnorm), _ptr(radius), float(alpha),
+                                   float(alpha_rescue), sink_blocks, window_blocks, _ptr(row_ptr),
+                                   _ptr(col_idx), cap, _ptr(nnz), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "fpx_select_rescue")
+    return row_ptr, col_idx, nnz
 
 
 def prefill(q, k, v, block: int, alpha: float, cu_seqlens=None, sink_blocks: int = 1,

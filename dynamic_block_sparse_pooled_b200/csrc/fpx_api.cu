@@ -195,8 +195,9 @@ int fpx_attention_path(const fpx_problem* p) {
 }
 
 static fpx_status block_scores_impl(const fpx_problem* p, const void* q, const void* k,
-                                    const fpx_paged_kv* kv, float* scores, void* ws,
-                                    size_t ws_bytes, fpx_stream_t stream) {
+                                    const fpx_paged_kv* kv, float* scores, float* qnorm,
+                                    float* radius, void* ws, size_t ws_bytes,
+                                    fpx_stream_t stream) {
   Sizes sz;
   fpx_status rc = check_problem(p, &sz);
   if (rc != FPX_OK) return rc;
@@ -222,30 +223,52 @@ static fpx_status block_scores_impl(const fpx_problem* p, const void* q, const v
     return FPX_ERR_CUDA;
   if (launch_score(d, p->dtype, qbar, kbar, qlo, klo, scores, t, st, s) != cudaSuccess)
     return FPX_ERR_CUDA;
+  if (qnorm && launch_radius(d, p->dtype, k, qbar, kbar, qlo, klo, qnorm, radius, t, s) !=
+                   cudaSuccess)
+    return FPX_ERR_CUDA;
   return FPX_OK;
 }
 
 fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, float* scores,
                             void* ws, size_t ws_bytes, fpx_stream_t stream) {
-  return block_scores_impl(p, q, k, nullptr, scores, ws, ws_bytes, stream);
+  return block_scores_impl(p, q, k, nullptr, scores, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+fpx_status fpx_block_scores_rescue(const fpx_problem* p, const void* q, const void* k,
+                                   const fpx_paged_kv* kv, float* scores, float* qnorm,
+                                   float* radius, void* ws, size_t ws_bytes,
+                                   fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if (sz.nb > 0 && (!qnorm || !radius)) return FPX_ERR_INVALID_ARG;
+  if (!aligned(qnorm, 4) || !aligned(radius, 4)) return FPX_ERR_ALIGNMENT;
+  return block_scores_impl(p, q, k, kv, scores, qnorm, radius, ws, ws_bytes, stream);
 }
 
 fpx_status fpx_block_scores_paged(const fpx_problem* p, const void* q, const void* k_cache,
                                   const fpx_paged_kv* kv, float* scores, void* ws,
                                   size_t ws_bytes, fpx_stream_t stream) {
   if (!kv) return FPX_ERR_INVALID_ARG;
-  return block_scores_impl(p, q, k_cache, kv, scores, ws, ws_bytes, stream);
+  return block_scores_impl(p, q, k_cache, kv, scores, nullptr, nullptr, ws, ws_bytes, stream);
 }
 
-fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, int32_t sink_blocks,
-                      int32_t window_blocks, int32_t* row_ptr, int32_t* col_idx,
-                      int64_t col_capacity, int64_t* nnz_d, void* ws, size_t ws_bytes,
-                      fpx_stream_t stream) {
+static fpx_status select_impl(const fpx_problem* p, const float* scores, const float* qnorm,
+                              const float* radius, float alpha, float alpha_rescue,
+                              int32_t sink_blocks, int32_t window_blocks, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int64_t* nnz_d, void* ws,
+                              size_t ws_bytes, fpx_stream_t stream) {
   Sizes sz;
   fpx_status rc = check_problem(p, &sz);
   if (rc != FPX_OK) return rc;
   if ((rc = check_ws(p, sz, 1, ws, ws_bytes)) != FPX_OK) return rc;
   if (std::isnan(alpha) || alpha < 0.f) return FPX_ERR_INVALID_ARG;
+  const bool rescue = qnorm != nullptr || radius != nullptr;
+  if (rescue) {
+    if (std::isnan(alpha_rescue) || alpha_rescue < 0.f) return FPX_ERR_INVALID_ARG;
+    if (sz.tri > 0 && (!qnorm || !radius)) return FPX_ERR_INVALID_ARG;
+    if (!aligned(qnorm, 4) || !aligned(radius, 4)) return FPX_ERR_ALIGNMENT;
+  }
   if (sink_blocks < 0 || window_blocks < 0 || col_capacity < 0) return FPX_ERR_INVALID_ARG;
   if (!row_ptr) return FPX_ERR_INVALID_ARG;
   if (sz.tri > 0 && (!scores || (!col_idx && col_capacity > 0))) return FPX_ERR_INVALID_ARG;
@@ -270,10 +293,32 @@ fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, in
   const int sink = sink_blocks > d.nb_total ? d.nb_total + 1 : sink_blocks;
   const int window = window_blocks > d.nb_total ? d.nb_total + 1 : window_blocks;
   if (launch_select(d, scores, alpha, sink, window, row_ptr, col_idx, col_capacity, nnz_d, rowmax,
-                    counts, cta_tot, overflow, mask, static_cast<int>(mask_words(sz)), t, st,
+                    counts, cta_tot, overflow, mask, static_cast<int>(mask_words(sz)),
+                    rescue ? qnorm : nullptr, rescue ? radius : nullptr, alpha_rescue, t, st,
                     s) != cudaSuccess)
     return FPX_ERR_CUDA;
   return FPX_OK;
+}
+
+fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha, int32_t sink_blocks,
+                      int32_t window_blocks, int32_t* row_ptr, int32_t* col_idx,
+                      int64_t col_capacity, int64_t* nnz_d, void* ws, size_t ws_bytes,
+                      fpx_stream_t stream) {
+  return select_impl(p, scores, nullptr, nullptr, alpha, 0.f, sink_blocks, window_blocks, row_ptr,
+                     col_idx, col_capacity, nnz_d, ws, ws_bytes, stream);
+}
+
+fpx_status fpx_select_rescue(const fpx_problem* p, const float* scores, const float* qnorm,
+                             const float* radius, float alpha, float alpha_rescue,
+                             int32_t sink_blocks, int32_t window_blocks, int32_t* row_ptr,
+                             int32_t* col_idx, int64_t col_capacity, int64_t* nnz_d, void* ws,
+                             size_t ws_bytes, fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if (sz.tri > 0 && (!qnorm || !radius)) return FPX_ERR_INVALID_ARG;
+  return select_impl(p, scores, qnorm, radius, alpha, alpha_rescue, sink_blocks, window_blocks,
+                     row_ptr, col_idx, col_capacity, nnz_d, ws, ws_bytes, stream);
 }
 
 static fpx_status sparse_prefill_impl(const fpx_problem* p, const void* q, const void* k,

@@ -31,8 +31,14 @@ cudaError_t launch_score_tc(const ProblemDesc& p, const float* qhi, const float*
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
                           int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
-                          int* overflow, uint32_t* mask, int mask_words, SeqTables t,
-                          StatusBlock* st, cudaStream_t s);
+                          int* overflow, uint32_t* mask, int mask_words, const float* qn,
+                          const float* rad, float alpha_r, SeqTables t, StatusBlock* st,
+                          cudaStream_t s);
+// Rescue-branch inputs after the pool pass: qnorm [Hq, NB] = ||qbar||, radius [Hkv, NB] = max
+// distance of a key of the block from its centroid (qlo / klo: the tf32 remainders, or null).
+cudaError_t launch_radius(const ProblemDesc& p, fpx_dtype dt, const void* k, const float* qbar,
+                          const float* kbar, const float* qlo, const float* klo, float* qnorm,
+                          float* radius, SeqTables t, cudaStream_t s);
 // CTAs of the select kernels (each owns 8 rows); the workspace holds one int64 per CTA.
 int select_ctas(const ProblemDesc& p);
 

@@ -264,6 +264,115 @@ cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const
 }
 
 // ------------------------------------------------------------------------------------------
+// rescue-branch inputs: radius[kvh * NB + b] = max over the block's valid rows j of
+// || k_j - kbar_b ||_2 (the largest distance of a key from its block centroid) and
+// qnorm[h * NB + b] = || qbar_b ||_2.  One warp per (block, head); D / 32 elements per lane.
+// ------------------------------------------------------------------------------------------
+constexpr int kRadWarps = 8;
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x) { return static_cast<float>(x); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_fp8_e4m3>(__nv_fp8_e4m3 x) { return static_cast<float>(x); }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kRadWarps * 32) radius_kernel(
+    ProblemDesc p, const T* __restrict__ k, const float* __restrict__ qbar,
+    const float* __restrict__ kbar, const float* __restrict__ qlo, const float* __restrict__ klo,
+    float* __restrict__ qnorm, float* __restrict__ radius, const int32_t* __restrict__ blk_base,
+    const int32_t* __restrict__ valid) {
+  constexpr int E = D / 32;  // elements per lane
+  if (!*valid) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t pair = static_cast<int64_t>(blockIdx.x) * kRadWarps + (threadIdx.x >> 5);
+  const int64_t n_k = static_cast<int64_t>(p.nb_total) * p.hkv;
+  const int64_t n_q = static_cast<int64_t>(p.nb_total) * p.hq;
+  if (pair >= n_k + n_q) return;
+  if (pair >= n_k) {  // query norm of pooled block b, head h
+    const int64_t qi = pair - n_k;
+    const int b = static_cast<int>(qi / p.hq), h = static_cast<int>(qi - static_cast<int64_t>(b) * p.hq);
+    const float* hi = qbar + (static_cast<int64_t>(b) * p.hq + h) * D;
+    const float* lo = qlo ? qlo + (static_cast<int64_t>(b) * p.hq + h) * D : nullptr;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float x = hi[lane * E + e] + (lo ? lo[lane * E + e] : 0.f);
+      acc = fmaf(x, x, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) qnorm[static_cast<int64_t>(h) * p.nb_total + b] = sqrtf(acc);
+    return;
+  }
+  const int b = static_cast<int>(pair / p.hkv), kvh = static_cast<int>(pair - static_cast<int64_t>(b) * p.hkv);
+  const int s = seq_of_block(blk_base, p.num_seqs, b);
+  const int I = b - blk_base[s];
+  const int rows = min(p.block, seq_len(p, s) - I * p.block);
+  const int64_t row0 = kv_block_row(p, s, I, seq_start(p, s));
+  float c[E];
+  {
+    const float* hi = kbar + (static_cast<int64_t>(b) * p.hkv + kvh) * D;
+    const float* lo = klo ? klo + (static_cast<int64_t>(b) * p.hkv + kvh) * D : nullptr;
+#pragma unroll
+    for (int e = 0; e < E; ++e) c[e] = hi[lane * E + e] + (lo ? lo[lane * E + e] : 0.f);
+  }
+  float best = 0.f;
+  if (row0 >= 0) {  // an invalid page was recorded by the pool kernel; its radius stays 0
+    const T* base = k + (row0 * p.hkv + kvh) * D + lane * E;
+    const int64_t stride = static_cast<int64_t>(p.hkv) * D;
+    for (int j0 = 0; j0 < rows; j0 += 4) {  // four rows in flight
+      float d2[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float acc = 0.f;
+        if (j0 + u < rows) {
+          const T* src = base + (j0 + u) * stride;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float x = to_f32<T>(src[e]) - c[e];
+            acc = fmaf(x, x, acc);
+          }
+        }
+        d2[u] = acc;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float a = d2[u];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        best = fmaxf(best, a);
+      }
+    }
+  }
+  if (lane == 0) radius[static_cast<int64_t>(kvh) * p.nb_total + b] = sqrtf(best);
+}
+
+cudaError_t launch_radius(const ProblemDesc& p, fpx_dtype dt, const void* k, const float* qbar,
+                          const float* kbar, const float* qlo, const float* klo, float* qnorm,
+                          float* radius, SeqTables t, cudaStream_t s) {
+  if (p.nb_total == 0) return cudaSuccess;
+  const int64_t pairs = static_cast<int64_t>(p.nb_total) * (p.hkv + p.hq);
+  const unsigned grid = static_cast<unsigned>((pairs + kRadWarps - 1) / kRadWarps);
+#define FPX_RAD(T, DD)                                                                        \
+  radius_kernel<T, DD><<<grid, kRadWarps * 32, 0, s>>>(p, static_cast<const T*>(k), qbar, kbar, \
+                                                       qlo, klo, qnorm, radius, t.blk_base,   \
+                                                       t.valid)
+  if (p.d == 128) {
+    if (dt == FPX_F32) FPX_RAD(float, 128);
+    else if (dt == FPX_BF16) FPX_RAD(__nv_bfloat16, 128);
+    else FPX_RAD(__nv_fp8_e4m3, 128);
+  } else {
+    if (dt == FPX_F32) FPX_RAD(float, 64);
+    else if (dt == FPX_BF16) FPX_RAD(__nv_bfloat16, 64);
+    else FPX_RAD(__nv_fp8_e4m3, 64);
+  }
+#undef FPX_RAD
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
 // score: one CTA per (64 x 64 tile of global block pairs (b, c) with c <= b, Q head); the tiles
 // of the lower triangle are enumerated by blockIdx.x.  A pair is written iff both blocks lie in
 // the same sequence and c <= b; tiles that hold no such pair return at once.
@@ -426,7 +535,8 @@ __device__ __forceinline__ float row_max_warp(const float* __restrict__ row, int
 __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
     ProblemDesc p, const float* __restrict__ scores, float alpha, int sink, int window,
     float* __restrict__ rowmax, int32_t* __restrict__ counts, int64_t* __restrict__ cta_tot,
-    uint32_t* __restrict__ mask, int mask_words, SeqTables t) {
+    uint32_t* __restrict__ mask, int mask_words, const float* __restrict__ qn,
+    const float* __restrict__ rad, float alpha_r, SeqTables t) {
   if (!*t.valid) return;
   __shared__ int w_tot[kSelWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -437,7 +547,34 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
     if (r >= R) break;
     const RowInfo ri = row_info(p, t, r);
     const float* row = scores + ri.base;
-    const float m = row_max_warp(row, ri.len, lane);
+    // rescue branch (qn != nullptr): u_J = s_J + scale_h * ||qbar_I|| * r_J, kept iff
+    // alpha_r == 0 or exp(u_J - max u) >= alpha_r, OR-ed with the base test
+    float m, mu = 0.f, cr = 0.f;
+    const float* radk = nullptr;
+    if (qn) {
+      const int h = r / p.nb_total, b = r - h * p.nb_total;
+      const int kvh = h / p.group;
+      const int first = t.blk_base[seq_of_block(t.blk_base, p.num_seqs, b)];
+      float sc = p.scale;
+      if (p.q_scale) sc *= p.q_scale[h] * p.k_scale[kvh];
+      cr = sc * qn[r];
+      radk = rad + static_cast<int64_t>(kvh) * p.nb_total + first;
+      float m0 = -CUDART_INF_F, u0 = -CUDART_INF_F;
+      for (int j = lane; j < ri.len; j += 32) {
+        const float v = row[j];
+        m0 = fmaxf(m0, v);
+        u0 = fmaxf(u0, fmaf(cr, radk[j], v));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        u0 = fmaxf(u0, __shfl_xor_sync(0xffffffffu, u0, o));
+      }
+      m = m0;
+      mu = u0;
+    } else {
+      m = row_max_warp(row, ri.len, lane);
+    }
     int cnt = 0;
     for (int j0 = 0; j0 < ri.len; j0 += 128) {  // four loads in flight per lane
       float v[4];
@@ -449,7 +586,9 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int j = j0 + 32 * u + lane;
-        const bool kp = j < ri.len && keep_block(v[u], m, alpha, j, ri.I, sink, window);
+        bool kp = j < ri.len && keep_block(v[u], m, alpha, j, ri.I, sink, window);
+        if (radk && j < ri.len && !kp)
+          kp = alpha_r == 0.f || expf(fmaf(cr, radk[j], v[u]) - mu) >= alpha_r;
         const unsigned bal = __ballot_sync(0xffffffffu, kp);
         const int w = (j0 >> 5) + u;
         if (lane == 0 && w < mask_words) mask[static_cast<int64_t>(r) * mask_words + w] = bal;
@@ -580,13 +719,15 @@ int select_ctas(const ProblemDesc& p) { return (p.hq * p.nb_total + kSelRows - 1
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
                           int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
-                          int* overflow, uint32_t* mask, int mask_words, SeqTables t,
-                          StatusBlock* st, cudaStream_t s) {
+                          int* overflow, uint32_t* mask, int mask_words, const float* qn,
+                          const float* rad, float alpha_r, SeqTables t, StatusBlock* st,
+                          cudaStream_t s) {
   const int R = p.hq * p.nb_total;
   const int nblk = select_ctas(p);
   if (R > 0) {
     select_count_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
-                                                       counts, cta_tot, mask, mask_words, t);
+                                                       counts, cta_tot, mask, mask_words, qn,
+                                                       rad, alpha_r, t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -182,6 +182,33 @@ fpx_status fpx_sparse_prefill_paged(const fpx_problem* p, const void* q, const v
                                     float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream);
 
 /*
+ * Radius rescue branch (the RBS-Attention abstract listed on the FlashPrefill page: a block
+ * centroid may hide a highly relevant token -- "mean dilution"; a rescue branch driven by the
+ * maximum key-block radius, thresholded independently and OR-ed with the centroid branch).  The
+ * page gives no formula; this library implements the Cauchy-Schwarz reading:
+ *   radius r_J = max over the valid tokens j of block J of || k_j - mean_J k ||_2 (per KV head),
+ *   u_IJ = s_IJ + scale * || mean_I q ||_2 * r_J  >= scale * <mean_I q, k_j> for every j in J,
+ *   rescue keep = alpha_rescue == 0 or exp(u_IJ - max_J' u_IJ') >= alpha_rescue (> 1: none),
+ *   final keep = the fpx_select keep OR the rescue keep (J <= I).
+ *
+ * fpx_block_scores_rescue: fpx_block_scores (kv NULL: packed K, else the paged cache of
+ *   fpx_block_scores_paged) that also writes qnorm fp32 [hq, NB] (h * NB + b: || mean q ||) and
+ *   radius fp32 [hkv, NB] (kvh * NB + b), reading K a second time.  Workspace: stage 0.
+ */
+fpx_status fpx_block_scores_rescue(const fpx_problem* p, const void* q, const void* k,
+                                   const fpx_paged_kv* kv, float* scores, float* qnorm,
+                                   float* radius, void* ws, size_t ws_bytes,
+                                   fpx_stream_t stream);
+
+/* fpx_select with the rescue branch OR-ed in; alpha_rescue >= 0 (NaN: FPX_ERR_INVALID_ARG).
+ * Same outputs, workspace (stage 1) and device-side conditions as fpx_select. */
+fpx_status fpx_select_rescue(const fpx_problem* p, const float* scores, const float* qnorm,
+                             const float* radius, float alpha, float alpha_rescue,
+                             int32_t sink_blocks, int32_t window_blocks, int32_t* row_ptr,
+                             int32_t* col_idx, int64_t col_capacity, int64_t* nnz_d, void* ws,
+                             size_t ws_bytes, fpx_stream_t stream);
+
+/*
  * Allocation-free variant of fpx_select (the paper has no counterpart; it exists for callers).
  *   Some callers cannot allocate device memory where they run: a plugin whose host framework
  *   owns all device memory and offers no scratch buffer, or latency-critical code that must not

@@ -154,3 +154,17 @@ def test_paged_argument_errors():
     pd, keep3 = make([300, 1000], d=64)
     assert lib.fpx_sparse_prefill_paged(ctypes.byref(pd), a, a, a, ctypes.byref(ok_kv), a, a, a,
                                         a, a, big, None) == -2
+
+
+def test_rescue_argument_errors():
+    lib = fpx.load()
+    p, keep = make([300])
+    ref = ctypes.byref(p)
+    big = 1 << 30
+    a = 0x100000
+    assert lib.fpx_block_scores_rescue(ref, a, a, None, a, None, a, a, big, None) == -1  # no qnorm
+    assert lib.fpx_block_scores_rescue(ref, a, a, None, a, a + 2, a, a, big, None) == -3
+    assert lib.fpx_select_rescue(ref, a, a, a, 0.1, float("nan"), 1, 1, a, a, 10, a, a, big,
+                                 None) == -1
+    assert lib.fpx_select_rescue(ref, a, a, a, 0.1, -1.0, 1, 1, a, a, 10, a, a, big, None) == -1
+    assert lib.fpx_select_rescue(ref, a, None, a, 0.1, 0.2, 1, 1, a, a, 10, a, a, big, None) == -1
