@@ -205,6 +205,57 @@ def sdpa_baseline(w, dev, cu, device, reps=2):
         return {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
 
 
+def extras(fpx, w, pf, dev, cu, ws, scores, row_ptr, col_idx, device, reps=3):
+    """Timings of the optional paths on the same inputs (after the timed region): attention with
+    K / V in a page cache (pages in reverse order) and the search with the radius rescue branch
+    (alpha_rescue 0.1).  Each is the mean of `reps` CUDA-event-timed calls after one warm-up."""
+    out = {}
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(device)
+        a, b = ev(), ev()
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        return round(a.elapsed_time(b) / reps, 4)
+
+    try:
+        if fpx.attention_path(pf) == 1:
+            nbs = [-(-(int(cu[i + 1]) - int(cu[i])) // w.block) for i in range(len(cu) - 1)]
+            npg = sum(nbs)
+            table = torch.full((len(nbs), max(1, max(nbs))), -1, dtype=torch.int32)
+            kc = torch.zeros((npg * w.block,) + tuple(dev["k"].shape[1:]), dtype=dev["k"].dtype,
+                             device=device)
+            vc = torch.zeros_like(kc)
+            pg = npg
+            for s_, nb in enumerate(nbs):
+                for J in range(nb):
+                    pg -= 1
+                    table[s_, J] = pg
+                    a_ = int(cu[s_]) + J * w.block
+                    b_ = min(int(cu[s_ + 1]), a_ + w.block)
+                    kc[pg * w.block: pg * w.block + (b_ - a_)] = dev["k"][a_:b_]
+                    vc[pg * w.block: pg * w.block + (b_ - a_)] = dev["v"][a_:b_]
+            kv = fpx.paged_kv(table.to(device), npg)
+            out["paged_attn_ms"] = timed(lambda: fpx.sparse_prefill_paged(
+                pf, dev["q"], kc, vc, kv, row_ptr, col_idx, ws))
+            del kc, vc
+
+        def rescue_search():
+            sc, qn, rad = fpx.block_scores_rescue(pf, dev["q"], dev["k"], ws)
+            fpx.select_rescue(pf, sc, qn, rad, w.alpha, 0.1, ws, w.sink_blocks, w.window_blocks)
+        out["rescue_search_ms"] = timed(rescue_search)
+        if fpx.status(ws) != 0:
+            return {"unavailable": f"device status {fpx.status(ws)}"}
+    except Exception as e:  # reported, never hidden
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
+    return out
+
+
 def run_ours(args, rank, world, device):
     import dynamic_block_sparse_pooled_b200 as fpx
 
@@ -338,6 +389,8 @@ def run_ours(args, rank, world, device):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "sdpa_baseline": sdpa_baseline(w, dev, cu, device) if not args.no_sdpa else None,
+        "extras": extras(fpx, w, pf, dev, cu, ws, scores, row_ptr, col_idx, device)
+        if not args.no_sdpa else None,
         "clocks": clk.summary(),
     }
     return res, w, data
@@ -427,7 +480,8 @@ def main():
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-sdpa", action="store_true", help="skip the PyTorch SDPA baseline")
+    ap.add_argument("--no-sdpa", action="store_true",
+                    help="skip the PyTorch SDPA baseline and the paged / rescue timings")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
