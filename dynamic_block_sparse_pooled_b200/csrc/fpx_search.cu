@@ -12,6 +12,12 @@
 //   * select_*      per query-block row: row max, the alpha test exp(s - m) >= alpha OR sink OR
 //                   window, warp ballot/popc compaction into CSR (no sort, no cumulative sum
 //                   over scores).
+// K may be read from a paged cache (FlashPrefill V2 abstract: paged KV cache): the pool kernel
+// then takes key block J of sequence s from its page (kv_block_row).
+// Radius rescue branch (RBS-Attention abstract: a rescue branch from the maximum key-block
+// radius, thresholded independently and OR-ed with the centroid branch):
+//   * radius_kernel max distance of a key from its block centroid, and the pooled query norms;
+//                   the select count pass then also tests u = s + scale * |qbar_I| * r_J.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
