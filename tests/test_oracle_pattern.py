@@ -1,0 +1,77 @@
+"""Pins of the query-probe vertical / slash oracle (oracle/pattern_oracle.py): probe placement,
+the dense limit against a library attention, planted vertical and slash structure, brute force
+of token-masked attention, threshold edge cases."""
+import numpy as np
+import torch
+
+from oracle import fpx_oracle as O
+from oracle import pattern_oracle as PO
+
+
+def test_probe_positions_are_uniform_and_end_at_the_last_token():
+    assert PO.probe_positions(100, 4).tolist() == [24, 49, 74, 99]
+    assert PO.probe_positions(5, 10).tolist() == [0, 1, 2, 3, 4]  # at most one probe per token
+    assert PO.probe_positions(7, 1).tolist() == [6]
+    assert PO.probe_positions(0, 4).size == 0
+
+
+def test_alpha_zero_is_dense_causal_attention():
+    rng = np.random.default_rng(0)
+    t, hq, hkv, d = 40, 2, 1, 8
+    q, k, v = (rng.standard_normal((t, h, d)) for h in (hq, hkv, hkv))
+    cu = [0, 15, 40]
+    found = PO.discover(q, k, cu, 4, 0.0, 0.5)
+    masks = [[PO.token_mask(n, vs[h], ss[h]) for h in range(hq)]
+             for n, (vs, ss) in zip([15, 25], found)]
+    o, lse = PO.attention_token_mask(q, k, v, cu, masks)
+    for a, b in ((0, 15), (15, 40)):
+        qq = torch.from_numpy(q[a:b]).permute(1, 0, 2)[None]
+        kk = torch.from_numpy(np.repeat(k[a:b], hq // hkv, axis=1)).permute(1, 0, 2)[None]
+        vv = torch.from_numpy(np.repeat(v[a:b], hq // hkv, axis=1)).permute(1, 0, 2)[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+        assert np.allclose(o[a:b], ref[0].permute(1, 0, 2).numpy(), atol=1e-12)
+
+
+def test_planted_vertical_and_slash_are_found():
+    rng = np.random.default_rng(1)
+    n, d, star, delta = 64, 16, 5, 3
+    base = rng.standard_normal(d)
+    q = (4.0 * base + 0.1 * rng.standard_normal((n, d)))[:, None, :]
+    k = 0.1 * rng.standard_normal((n, 1, d))
+    k[star, 0] = 3.0 * base  # every query attends token `star`
+    verts, _ = PO.discover(q, k, [0, n], 8, 0.5, 2.0)[0]
+    assert star in verts[0]
+    # slash: key j points at query j + delta, so every query's best key sits `delta` back
+    q2 = rng.standard_normal((n, 1, d)) * 3.0
+    k2 = 0.1 * rng.standard_normal((n, 1, d))
+    k2[:n - delta, 0] = q2[delta:, 0]
+    _, slashes = PO.discover(q2, k2, [0, n], 8, 2.0, 0.9)[0]
+    assert delta in slashes[0]
+    mask = PO.token_mask(n, np.zeros(0, int), slashes[0])
+    assert all(mask[i, i - delta] for i in range(delta, n))
+    assert not any(mask[i, i + 1] for i in range(n - 1))  # causal
+
+
+def test_token_masked_attention_matches_brute_force():
+    rng = np.random.default_rng(2)
+    n, d = 12, 4
+    q, k, v = (rng.standard_normal((n, 1, d)) for _ in range(3))
+    verts, slashes = np.array([0, 7]), np.array([0, 2])
+    mask = PO.token_mask(n, verts, slashes)
+    o, lse = PO.attention_token_mask(q, k, v, [0, n], [[mask]])
+    sc = 1.0 / np.sqrt(d)
+    for i in range(n):
+        js = [j for j in range(i + 1) if j in verts or (i - j) in slashes]
+        lg = np.array([sc * q[i, 0] @ k[j, 0] for j in js])
+        w = np.exp(lg - lg.max())
+        assert np.allclose(o[i, 0], (w[:, None] * v[js, 0]).sum(0) / w.sum())
+        assert np.isclose(lse[0, i], lg.max() + np.log(w.sum()))
+
+
+def test_threshold_edges():
+    rng = np.random.default_rng(3)
+    q, k = rng.standard_normal((20, 2, 4)), rng.standard_normal((20, 1, 4))
+    verts, slashes = PO.discover(q, k, [0, 20], 5, 1.5, 1.5)[0]
+    assert all(x.size == 0 for x in verts) and all(x.size == 0 for x in slashes)
+    verts, slashes = PO.discover(q, k, [0, 20], 5, 1.0, 1.0)[0]
+    assert all(x.size >= 1 for x in verts) and all(x.size >= 1 for x in slashes)  # the maxima
