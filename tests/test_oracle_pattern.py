@@ -8,14 +8,14 @@ from oracle import fpx_oracle as O
 from oracle import pattern_oracle as PO
 
 
-def test_probe_positions_are_uniform_and_end_at_the_last_token():
+def check_probe_positions_are_uniform_and_end_at_the_last_token(PO=PO):
     assert PO.probe_positions(100, 4).tolist() == [24, 49, 74, 99]
     assert PO.probe_positions(5, 10).tolist() == [0, 1, 2, 3, 4]  # at most one probe per token
     assert PO.probe_positions(7, 1).tolist() == [6]
     assert PO.probe_positions(0, 4).size == 0
 
 
-def test_alpha_zero_is_dense_causal_attention():
+def check_alpha_zero_is_dense_causal_attention(PO=PO):
     rng = np.random.default_rng(0)
     t, hq, hkv, d = 40, 2, 1, 8
     q, k, v = (rng.standard_normal((t, h, d)) for h in (hq, hkv, hkv))
@@ -32,7 +32,7 @@ def test_alpha_zero_is_dense_causal_attention():
         assert np.allclose(o[a:b], ref[0].permute(1, 0, 2).numpy(), atol=1e-12)
 
 
-def test_planted_vertical_and_slash_are_found():
+def check_planted_vertical_and_slash_are_found(PO=PO):
     rng = np.random.default_rng(1)
     n, d, star, delta = 64, 16, 5, 3
     base = rng.standard_normal(d)
@@ -52,7 +52,7 @@ def test_planted_vertical_and_slash_are_found():
     assert not any(mask[i, i + 1] for i in range(n - 1))  # causal
 
 
-def test_token_masked_attention_matches_brute_force():
+def check_token_masked_attention_matches_brute_force(PO=PO):
     rng = np.random.default_rng(2)
     n, d = 12, 4
     q, k, v = (rng.standard_normal((n, 1, d)) for _ in range(3))
@@ -68,10 +68,54 @@ def test_token_masked_attention_matches_brute_force():
         assert np.isclose(lse[0, i], lg.max() + np.log(w.sum()))
 
 
-def test_threshold_edges():
+def check_threshold_edges(PO=PO):
     rng = np.random.default_rng(3)
     q, k = rng.standard_normal((20, 2, 4)), rng.standard_normal((20, 1, 4))
     verts, slashes = PO.discover(q, k, [0, 20], 5, 1.5, 1.5)[0]
     assert all(x.size == 0 for x in verts) and all(x.size == 0 for x in slashes)
     verts, slashes = PO.discover(q, k, [0, 20], 5, 1.0, 1.0)[0]
     assert all(x.size >= 1 for x in verts) and all(x.size >= 1 for x in slashes)  # the maxima
+
+
+def check_aggregation_over_probes_is_the_max(PO=PO):
+    # probe rows given directly: key 0 gets 0.6 from one probe, key 1 gets 0.35 from three;
+    # the max reading keeps key 0 (a sum would prefer key 1); offsets likewise
+    a = np.zeros((1, 3, 4))
+    a[0, 0, :2] = [0.6, 0.4]            # probe at position 1
+    a[0, 1, :3] = [0.3, 0.35, 0.35]     # probe at position 2
+    a[0, 2, :4] = [0.3, 0.35, 0.0, 0.35]  # probe at position 3
+    verts, slashes = PO.vertical_slash(a, np.array([1, 2, 3]), 0.9, 0.9)
+    assert verts[0].tolist() == [0]
+    # slash offsets: probe 1 -> {0: 0.4, 1: 0.6}; probe 2 -> {0: .35, 1: .35, 2: .3};
+    # probe 3 -> {0: .35, 1: 0, 2: .35, 3: .3}: max per offset 0.4, 0.6, 0.35, 0.3
+    assert slashes[0].tolist() == [1]
+
+
+ALL_CHECKS = [check_probe_positions_are_uniform_and_end_at_the_last_token,
+              check_alpha_zero_is_dense_causal_attention, check_planted_vertical_and_slash_are_found,
+              check_token_masked_attention_matches_brute_force, check_threshold_edges,
+              check_aggregation_over_probes_is_the_max]
+
+
+def test_probe_positions_are_uniform_and_end_at_the_last_token():
+    check_probe_positions_are_uniform_and_end_at_the_last_token()
+
+
+def test_alpha_zero_is_dense_causal_attention():
+    check_alpha_zero_is_dense_causal_attention()
+
+
+def test_planted_vertical_and_slash_are_found():
+    check_planted_vertical_and_slash_are_found()
+
+
+def test_token_masked_attention_matches_brute_force():
+    check_token_masked_attention_matches_brute_force()
+
+
+def test_threshold_edges():
+    check_threshold_edges()
+
+
+def test_aggregation_over_probes_is_the_max():
+    check_aggregation_over_probes_is_the_max()
