@@ -39,9 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNELS_PER_STEP = 10  # plan+pool+score, plan+count+scan+emit, plan+order+attention
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch per workload,
-# from an ncu capture of the kernel built from sources whose digest is ATTN_TRAFFIC_DIGEST
-# (profiles/attn_tc_kernel_dram.md).  Reported as roofline.traffic only while the sources still
-# have that digest; any change to the kernel makes it null until it is measured again.
+# from an ncu capture of the kernel built from sources whose digest is ATTN_TRAFFIC_DIGEST.
+# Reported as roofline.traffic only while the sources still have that digest; any change to the
+# kernel makes it null until it is measured again.
 ATTN_SOURCES = ("dynamic_block_sparse_pooled_b200/csrc/fpx_attn_sm100.cu",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_sm100.cuh",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_common.cuh")
@@ -94,6 +94,15 @@ def aggregate_value(flops_per_rank: float, world: int, ms_per_step: float) -> fl
     """Whole-job dense-equivalent TFLOP/s: every rank runs its own prefill (weak scaling), the
     step time is the slowest rank's."""
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def config_of(w, world: int) -> dict:
+    """The workload description both arms print (same keys, same values)."""
+    return {"workload": w.name, "seqlens": list(w.seqlens), "hq": w.hq, "hkv": w.hkv,
+            "d": w.d, "block": w.block, "alpha": w.alpha, "sink_blocks": w.sink_blocks,
+            "window_blocks": w.window_blocks,
+            "l2": "inputs (Q+K+V) larger than L2; no flush",
+            "parallelism": f"replica x{world} (independent prefills)"}
 
 
 def dense_flops(w) -> float:
@@ -354,9 +363,11 @@ def run_ours(args, rank, world, device):
     if w.dtype == "e4m3":
         peak_tf *= 2.0  # fp8 dense is twice bf16 (nominal ratio)
     achieved = exec_flops / (attn_avg * 1e-3) / 1e12
+    # algorithmic bytes of the search: Q and K read once, the pooled scores written once, the CSR
+    # written (the select pass's read-back of the scores is reported apart, not counted)
     search_bytes = (dev["q"].numel() * dev["q"].element_size() +
                     dev["k"].numel() * dev["k"].element_size() +
-                    2 * 4 * w.hq * tri + 4 * (pf.rows + 1) + 4 * n_kept)
+                    4 * w.hq * tri + 4 * (pf.rows + 1) + 4 * n_kept)
     res = {
         "metric": METRIC,
         "value": round(aggregate_value(flops, world, ms_step), 3),
@@ -365,15 +376,12 @@ def run_ours(args, rank, world, device):
         "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded generator: RoPE + sink + verticals + slash)",
-        "config": {"workload": w.name, "seqlens": list(w.seqlens), "hq": w.hq, "hkv": w.hkv,
-                   "d": w.d, "block": w.block, "alpha": w.alpha, "sink_blocks": w.sink_blocks,
-                   "window_blocks": w.window_blocks,
-                   "l2": "inputs (Q+K+V) larger than L2; no flush",
-                   "parallelism": f"replica x{world} (independent prefills)"},
+        "config": config_of(w, world),
         "attn_ms": round(attn_avg, 4),
         "search_ms": round(statistics.mean(search_ms), 4),
         "attn_dense_equiv_tflops": round(flops / (attn_avg * 1e-3) / 1e12, 3),
         "density": round(density, 6), "nnz": n_kept,
+        "search_bytes": search_bytes, "search_scores_readback_bytes": 4 * w.hq * tri,
         "search_gbs": round(search_bytes / (statistics.mean(search_ms) * 1e-3) / 1e9, 1),
         "search_hbm_frac": round(search_bytes / (statistics.mean(search_ms) * 1e-3) / 1e9
                                  / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), 4),
@@ -454,17 +462,22 @@ def run_reference(args):
     for _ in range(args.warmup):
         oracle_sample(w, data, budget)
     vals = []
+    secs = []
     text = ""
     for _ in range(args.steps):
         flop, dt, text = oracle_sample(w, data, budget)
         vals.append(flop / dt / 1e12)
+        secs.append(dt)
     v = statistics.mean(vals)
     unit = "TFLOP/s (dense-equivalent causal attention, whole step)"
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * statistics.mean(secs), 3),
+        "ms_per_step_note": "wall time of one bounded oracle sample (see cpu_baseline.sample)",
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name},
+        "config": config_of(w, 1),
         "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                          "sample": text},
         "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -486,8 +499,20 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: relaunch this command under torchrun on this node
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+               f"--master-port={os.environ.get('MASTER_PORT', '29517')}",
+               os.path.abspath(__file__)] + sys.argv[1:]
+        import subprocess
+        sys.exit(subprocess.call(cmd))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

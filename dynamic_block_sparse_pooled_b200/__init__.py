@@ -31,7 +31,8 @@ EXPORTS = ("fpx_num_blocks", "fpx_scores_elems", "fpx_rows", "fpx_max_nnz", "fpx
            "fpx_clear_status", "fpx_query_status", "fpx_status_string", "fpx_block_scores",
            "fpx_select", "fpx_sparse_prefill", "fpx_attention_path", "fpx_select_noalloc",
            "fpx_select_noalloc_max_bytes", "fpx_diag_bounded_wait", "fpx_block_scores_paged",
-           "fpx_sparse_prefill_paged", "fpx_block_scores_rescue", "fpx_select_rescue")
+           "fpx_sparse_prefill_paged", "fpx_block_scores_rescue", "fpx_select_rescue",
+           "fpx_diag_exp2")
 
 
 class FpxError(RuntimeError):
@@ -105,6 +106,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fpx_select_noalloc_max_bytes.restype = sz
     lib.fpx_diag_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
     lib.fpx_diag_bounded_wait.restype = ctypes.c_int
+    lib.fpx_diag_exp2.argtypes = [vp, vp, i64, vp]
+    lib.fpx_diag_exp2.restype = ctypes.c_int
     K = ctypes.POINTER(PagedKV)
     lib.fpx_block_scores_paged.argtypes = [P, vp, vp, K, vp, vp, sz, vp]
     lib.fpx_block_scores_paged.restype = ctypes.c_int
@@ -212,6 +215,22 @@ def block_scores(pf: Prefill, q: torch.Tensor, k: torch.Tensor, ws: torch.Tensor
     return scores
 
 
+def _check_csr_outputs(pf: Prefill, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                       nnz: torch.Tensor, capacity: int) -> None:
+    """The library writes up to `capacity` col_idx entries and R + 1 row_ptr entries: refuse
+    buffers that cannot hold them (the device would write past the tensors)."""
+    if row_ptr.dtype != torch.int32 or col_idx.dtype != torch.int32 or nnz.dtype != torch.int64:
+        raise ValueError("row_ptr and col_idx must be int32 and nnz int64")
+    if not (row_ptr.is_contiguous() and col_idx.is_contiguous()):
+        raise ValueError("row_ptr and col_idx must be contiguous")
+    if row_ptr.numel() < pf.rows + 1:
+        raise ValueError(f"row_ptr holds {row_ptr.numel()} entries, needs {pf.rows + 1}")
+    if capacity < 0 or capacity > col_idx.numel():
+        raise ValueError(f"capacity {capacity} exceeds col_idx ({col_idx.numel()} entries)")
+    if nnz.numel() < 1:
+        raise ValueError("nnz needs one int64 entry")
+
+
 def select(pf: Prefill, scores: torch.Tensor, alpha: float, ws: torch.Tensor,
            sink_blocks: int = 1, window_blocks: int = 1, row_ptr=None, col_idx=None,
            nnz=None, capacity: Optional[int] = None, stream=None):
@@ -225,6 +244,7 @@ def select(pf: Prefill, scores: torch.Tensor, alpha: float, ws: torch.Tensor,
     cap = col_idx.numel() if capacity is None else capacity
     if nnz is None:
         nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    _check_csr_outputs(pf, row_ptr, col_idx, nnz, cap)
     check(load().fpx_select(pf.ptr, _ptr(scores), float(alpha), sink_blocks, window_blocks,
                             _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz), _ptr(ws), ws.numel(),
                             _stream(stream)), "fpx_select")
@@ -245,6 +265,7 @@ def select_noalloc(pf: Prefill, scores: torch.Tensor, alpha: float, sink_blocks:
     cap = col_idx.numel() if capacity is None else capacity
     if nnz is None:
         nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    _check_csr_outputs(pf, row_ptr, col_idx, nnz, cap)
     check(load().fpx_select_noalloc(pf.ptr, _ptr(scores), float(alpha), sink_blocks,
                                     window_blocks, _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz),
                                     _stream(stream)), "fpx_select_noalloc")

@@ -1,5 +1,5 @@
-"""Fits the polynomial behind the FMA-pipe exp2 used by the attention softmax (exp2_poly in
-fpx_attn_sm100.cu) and prints its coefficients and error bound.
+"""Fits the polynomial behind the FMA-pipe exp2 used by the attention softmax (exp2_poly2 in
+fpx_sm100.cuh) and prints its coefficients and error bound.
 
 Method: Cody-Waite style range reduction x = n + f with n = round(x), |f| <= 1/2, so that
 2^x = 2^n * 2^f; 2^n is applied by adding n to the exponent field.  2^f on [-1/2, 1/2] is a

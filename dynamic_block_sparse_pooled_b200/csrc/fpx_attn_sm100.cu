@@ -141,28 +141,6 @@ __device__ __forceinline__ float row_max64(const uint32_t* r) {
                fmaxf(__uint_as_float(r[62]), __uint_as_float(r[63])));
 }
 
-// 2^x on the FMA pipe, for x <= 128 (x below -126 flushes towards 0).  Cody-Waite style split
-// x = n + f, n = round(x) via the 1.5 * 2^23 shifter (the low bits of t then hold n), |f| <= 1/2;
-// 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative error on
-// [-1/2, 1/2] (Remez exchange; fitted by exp2_poly_fit.py, max relative error 7.5e-5, below
-// bf16 and e4m3 rounding of P); 2^n is added in the exponent field.
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f;
-  constexpr float C2 = 0.2426111251115799f, C3 = 0.0551716685295105f;
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  float t0, t1, n0, n1, f0, f1, p0, p1;
-  fadd2(t0 = x0, t1 = x1, kShift, kShift);
-  fadd2(n0 = t0, n1 = t1, -kShift, -kShift);
-  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
-  ffma2(p0, p1, C3, C3, f0, f1, C2, C2);
-  ffma2(p0, p1, p0, p1, f0, f1, C1, C1);
-  ffma2(p0, p1, p0, p1, f0, f1, C0, C0);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 // One in kPolyEvery element pairs takes exp2 on the FMA pipe instead of the MUFU (0: none).  The
 // MUFU issues four ex2 per cycle per SM sub-partition, so a 128-column row costs ~1000 cycles
 // there; moving a quarter of the pairs to the FMA pipe was measured fastest (one in two or three

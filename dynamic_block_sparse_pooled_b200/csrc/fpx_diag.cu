@@ -1,6 +1,11 @@
-// fpx_diag.cu -- fpx_diag_bounded_wait: exercises the bounded device-side wait that every
-// pipeline barrier of the library uses, on a barrier phase that nothing completes.
+// fpx_diag.cu -- diagnostics with no counterpart in the paper:
+//   fpx_diag_bounded_wait  exercises the bounded device-side wait that every pipeline barrier
+//                          of the library uses, on a barrier phase that nothing completes;
+//   fpx_diag_exp2          evaluates the FMA-pipe exp2 that the attention softmax applies to a
+//                          share of its elements, so that its error can be tested directly.
 #include <cuda_runtime.h>
+
+#include <climits>
 
 #include "fpx_internal.h"
 #include "fpx_sm100.cuh"
@@ -25,7 +30,29 @@ __global__ void bounded_wait_kernel(StatusBlock* st, uint64_t limit_ns) {
   if (done && threadIdx.x == 0) record_error(st, FPX_ERR_TIMEOUT, 40);
 }
 
+// y[i] = exp2_poly2(x[i]) (pairs of elements, as the softmax evaluates them).
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float y0, y1;
+  sm100::exp2_poly2(y0, y1, x0, x1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace fpx
+
+extern "C" fpx_status fpx_diag_exp2(const float* x, float* y, int64_t n, fpx_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return FPX_ERR_INVALID_ARG;
+  if (n == 0) return FPX_OK;
+  const int64_t pairs = (n + 1) / 2;
+  const int64_t blocks = (pairs + 255) / 256;
+  if (blocks > INT32_MAX) return FPX_ERR_UNSUPPORTED;
+  fpx::exp2_poly_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? FPX_OK : FPX_ERR_CUDA;
+}
 
 extern "C" fpx_status fpx_diag_bounded_wait(void* ws, uint64_t limit_ns, fpx_stream_t stream) {
   if (!ws) return FPX_ERR_INVALID_ARG;

@@ -25,22 +25,29 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
 // Host code must not use g_select_scratch's name as an address: on the host it is only a
-// stand-in for the device symbol.  The device address is looked up once per device, with that
-// device current, and cached.
-std::once_flag g_once[kMaxDevices];
+// stand-in for the device symbol.  The device address is looked up with the device current and
+// kept once a lookup has succeeded; a failed lookup (e.g. attempted inside a stream capture) is
+// not kept, so the next call tries again.
+std::mutex g_mu;
 void* g_addr[kMaxDevices];
-cudaError_t g_err[kMaxDevices];
 
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev] {
-    g_err[dev] = cudaGetSymbolAddress(&g_addr[dev], g_select_scratch);
-  });
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_addr[dev] == nullptr) {
+    void* a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_select_scratch);
+    if (e != cudaSuccess || a == nullptr) {
+      cudaGetLastError();  // do not leave the failed lookup as the thread's sticky-looking error
+      return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+    }
+    g_addr[dev] = a;
+  }
   *out = g_addr[dev];
-  return g_err[dev];
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -490,7 +490,8 @@ cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, con
 // select: a CTA owns 8 consecutive rows r = (h, s, I) (warp per row).
 //   count: row max, kept-block count per row, CTA total, and the row's keep bitmask (bit J of
 //          word J / 32 at mask[r * mask_words + J / 32]: the ballot of the keep test)
-//   scan:  exclusive scan of the CTA totals (one CTA), nnz, capacity check
+//   scan:  exclusive scan of the CTA totals (one CTA), nnz, capacity check (on overflow: an
+//          empty CSR, row_ptr all zero)
 //   emit:  per-CTA exclusive scan of its counts -> row_ptr; the bitmask (1/32 of the scores'
 //          bytes) compacted into col_idx with popc prefixes
 // ------------------------------------------------------------------------------------------
@@ -662,14 +663,24 @@ __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
     cta_tot[i] = run;  // in place: exclusive offsets
     run += c;
   }
+  const int64_t total = warp_tot[31];
+  if (total > capacity) {
+    // col_idx cannot hold the selection: publish an empty CSR (every row_ptr entry 0), so that
+    // no reader of (row_ptr, col_idx) can index past the capacity; nnz_d reports the count the
+    // caller would need, and the emit kernel writes nothing.
+    for (int i = tid; i <= R; i += kScanThreads) row_ptr[i] = 0;
+    if (tid == 0) {
+      if (nnz_d) *nnz_d = total;
+      *overflow = 1;
+      record_error(st, FPX_ERR_CAPACITY, 10, static_cast<int>(total >> 32),
+                   static_cast<int>(total & 0xffffffff));
+    }
+    return;
+  }
   if (tid == kScanThreads - 1) {
-    const int64_t total = warp_tot[31];
     row_ptr[R] = static_cast<int32_t>(total);
     if (nnz_d) *nnz_d = total;
-    const bool over = total > capacity;
-    *overflow = over ? 1 : 0;
-    if (over) record_error(st, FPX_ERR_CAPACITY, 10, static_cast<int>(total >> 32),
-                           static_cast<int>(total & 0xffffffff));
+    *overflow = 0;
   }
 }
 
@@ -678,7 +689,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
     int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
     const int* __restrict__ overflow, const uint32_t* __restrict__ mask, int mask_words,
     SeqTables t) {
-  if (!*t.valid) return;
+  if (!*t.valid || *overflow) return;  // the scan published an empty CSR
   __shared__ int32_t s_off[kSelRows];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int R = p.hq * p.nb_total;
@@ -698,7 +709,6 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
   const int64_t base = cta_off[blockIdx.x];
   if (threadIdx.x < kSelRows && r0 + threadIdx.x < R)
     row_ptr[r0 + threadIdx.x] = static_cast<int32_t>(base + s_off[threadIdx.x]);
-  if (*overflow) return;
   for (int k = 0; k < kSelRowsPerWarp; ++k) {
     const int rl = warp * kSelRowsPerWarp + k;
     const int r = r0 + rl;

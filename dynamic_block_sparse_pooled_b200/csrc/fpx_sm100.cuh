@@ -1,5 +1,6 @@
 // fpx_sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the attention mainloop
-// uses: mbarriers, TMA tensor loads, tcgen05 MMA / TMEM allocation / TMEM loads and stores.
+// uses: mbarriers, TMA tensor loads, tcgen05 MMA / TMEM allocation / TMEM loads and stores,
+// packed f32x2 arithmetic, and the FMA-pipe exp2 of the softmax.
 #pragma once
 
 #include <cuda.h>
@@ -233,6 +234,30 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) 
       "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "+f"(d0), "+f"(d1)
       : "f"(a0), "f"(a1));
+}
+
+// 2^x on the FMA pipe, for x <= 128; x below -125 is raised to -125 (2^-125 ~ 2.4e-38: a
+// weight that vanishes against any softmax row sum).  Cody-Waite style split x = n + f,
+// n = round(x) via the 1.5 * 2^23 shifter (the low bits of t then hold n), |f| <= 1/2; 2^f by a
+// degree-3 polynomial whose coefficients minimise the maximum relative error on [-1/2, 1/2]
+// (Remez exchange; fitted by exp2_poly_fit.py, max relative error 7.5e-5, below bf16 and e4m3
+// rounding of P); 2^n is added in the exponent field.  The clamp keeps that sum a normal number:
+// with n >= -125 and 2^f >= 0.7 the exponent field stays >= 1.
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f;
+  constexpr float C2 = 0.2426111251115799f, C3 = 0.0551716685295105f;
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0 = x0, t1 = x1, kShift, kShift);
+  fadd2(n0 = t0, n1 = t1, -kShift, -kShift);
+  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
+  ffma2(p0, p1, C3, C3, f0, f1, C2, C2);
+  ffma2(p0, p1, p0, p1, f0, f1, C1, C1);
+  ffma2(p0, p1, p0, p1, f0, f1, C0, C0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 // ---- descriptors ------------------------------------------------------------------------

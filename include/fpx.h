@@ -123,8 +123,11 @@ fpx_status fpx_block_scores(const fpx_problem* p, const void* q, const void* k, 
  *   alpha >= 0 (NaN rejected); sink_blocks, window_blocks >= 0.
  *   row_ptr   device int32 [R + 1], written (row_ptr[0] = 0, row_ptr[R] = nnz).
  *   col_idx   device int32 [col_capacity]; kept J per row, ascending.  If nnz > col_capacity
- *             nothing is written to col_idx and FPX_ERR_CAPACITY is recorded in the status.
- *   nnz_d     device int64 [1] (may be NULL): total kept blocks.
+ *             nothing is written to col_idx, row_ptr is written all zero (an empty CSR, which
+ *             fpx_sparse_prefill reads as rows with no key) and FPX_ERR_CAPACITY is recorded in
+ *             the status.
+ *   nnz_d     device int64 [1] (may be NULL): total kept blocks (on overflow: the capacity the
+ *             selection needs).
  *   ws        device workspace >= fpx_workspace_bytes(p, 1).
  */
 fpx_status fpx_select(const fpx_problem* p, const float* scores, float alpha,
@@ -222,11 +225,14 @@ fpx_status fpx_select_rescue(const fpx_problem* p, const float* scores, const fl
  *   160,000 rows Hq * NB when no sequence exceeds 32 blocks, about 28,000 at 512 blocks);
  *   larger problems return FPX_ERR_CAPACITY before anything is launched.  An invalid or unsupported problem returns FPX_ERR_INVALID_ARG.
  *   Device-side conditions are visible through the outputs: nnz > col_capacity means nothing was
- *   written to col_idx; device cu_seqlens that disagree with the host mirror give an empty CSR.
- *   The first call on a device looks up the array's device address (once per device, with that
- *   device current); make that first call before any stream capture.  All calls on a device
- *   share the array and each call re-zeroes the part that must start at zero: calls whose work
- *   overlaps on the GPU (unordered streams) race on it.
+ *   written to col_idx and row_ptr is all zero; device cu_seqlens that disagree with the host
+ *   mirror give an empty CSR with nnz 0.
+ *   The first successful call on a device looks up the array's device address (with that device
+ *   current) and keeps it for the life of the process; a failed lookup is retried by the next
+ *   call.  Make that first call before any stream capture.  A cudaDeviceReset after it is not
+ *   supported (the kept address would be stale).  All calls on a device share the array and each
+ *   call re-zeroes the part that must start at zero: calls whose work overlaps on the GPU
+ *   (unordered streams) race on it.
  */
 fpx_status fpx_select_noalloc(const fpx_problem* p, const float* scores, float alpha,
                               int32_t sink_blocks, int32_t window_blocks, int32_t* row_ptr,
@@ -242,6 +248,15 @@ size_t fpx_select_noalloc_max_bytes(void);
  * 256-byte aligned); the CUDA context stays usable.  Returns a launch status only.
  */
 fpx_status fpx_diag_bounded_wait(void* ws, uint64_t limit_ns, fpx_stream_t stream);
+
+/*
+ * Diagnostic (the paper has no counterpart): y[i] = 2^x[i] evaluated with the FMA-pipe
+ * exponential that fpx_sparse_prefill's softmax uses for a share of its elements (range
+ * reduction x = n + f, |f| <= 1/2, a degree-3 minimax polynomial for 2^f, n added to the
+ * exponent field).  Relative error <= 7.5e-5 for -125 <= x <= 8 (the softmax's range); x below
+ * -125 gives 2^-125 * 2^0 (a vanishing weight).  x, y: device fp32 [n].  Returns a launch status.
+ */
+fpx_status fpx_diag_exp2(const float* x, float* y, int64_t n, fpx_stream_t stream);
 
 /* Which attention kernel fpx_sparse_prefill uses for this problem: 1 = the tcgen05/TMEM
  * tensor-core mainloop (bf16 / e4m3, B = 128, D = 128), 0 = the CUDA-core kernel (fp32 and the

@@ -282,3 +282,75 @@ def check_block_evaluation_matches_full(O):
 
 
 ALL_CHECKS.append(check_block_evaluation_matches_full)
+
+
+def check_near_band_is_exactly_the_unforced_ratios_within_the_band(O):
+    """Hand-made score rows with known ratios exp(s - m): the near-threshold band must be exactly
+    the causal, not forced (sink / window) blocks whose ratio lies within 1e-3 * alpha of alpha
+    (the reporting rule for blocks whose decision rounding may flip).  Ratios sit at +-5e-4,
+    -9e-4 (inside) and +-2e-3 (outside) relative to alpha; the sink and diagonal blocks are put
+    inside the band to show that forced blocks are never reported."""
+    nb, hq = 8, 2
+    inside = {2: 1 + 5e-4, 3: 1 - 9e-4, 6: 1 - 5e-4}
+    outside = {4: 1 + 2e-3, 5: 1 - 2e-3}
+    for alpha in (0.05, 0.3, 0.9):
+        s = np.full((hq, nb, nb), -np.inf)
+        for h in range(hq):
+            c = 0.37 - 1.3 * h  # a per-row offset cancels in s - max s
+            for I in range(nb):
+                for J in range(I + 1):
+                    if J == I and I >= 2:
+                        r = alpha * (1 + 1e-4)        # diagonal: forced, inside the band
+                    elif J == 0 and I >= 1:
+                        r = alpha * (1 - 1e-4)        # sink: forced, inside the band
+                    elif J == 1 or I == 0:
+                        r = 1.0                       # the row maximum
+                    else:
+                        r = alpha * {**inside, **outside}[J]
+                    s[h, I, J] = c + math.log(r)
+        keeps, nears = O.select([s], alpha, 1, 1)
+        for h in range(hq):
+            for I in range(nb):
+                want_near = sorted(J for J in inside if J < I)
+                want_keep = sorted({0, 1, I} & set(range(I + 1)) | {J for J in (2, 4) if J < I})
+                assert np.nonzero(nears[0][h, I])[0].tolist() == want_near, (alpha, h, I)
+                assert np.nonzero(keeps[0][h, I])[0].tolist() == want_keep, (alpha, h, I)
+    keeps, nears = O.select([s], 0.0, 1, 1)  # alpha = 0: every causal block, nothing near
+    assert not nears[0].any()
+    assert np.array_equal(keeps[0], np.broadcast_to(np.tril(np.ones((nb, nb), bool)), s.shape))
+
+
+def check_triangular_pack_matches_the_layout_formula(O):
+    """Element (h, s, I, J <= I) of the packed scores sits at h * TRI + tri_base[s] + I (I + 1) / 2
+    + J, tri_base[s] = sum over earlier sequences of nb (nb + 1) / 2 (the C ABI's score layout),
+    checked on a varlen batch with ragged tails and a zero-length sequence."""
+    seqlens, block, hq = [130, 0, 64, 1, 257], 64, 3
+    nbs = [-(-n // block) for n in seqlens]
+    tri_base, acc = [], 0
+    for nb in nbs:
+        tri_base.append(acc)
+        acc += nb * (nb + 1) // 2
+    tri = acc
+    sc = []
+    for si, nb in enumerate(nbs):
+        a = np.full((hq, nb, nb), -np.inf)
+        for h in range(hq):
+            for I in range(nb):
+                for J in range(I + 1):
+                    a[h, I, J] = h * 1e6 + si * 1e4 + I * 100 + J
+        sc.append(a)
+    flat = np.asarray(O.triangular_pack(sc)).reshape(-1)
+    assert flat.size == hq * tri
+    seen = 0
+    for h in range(hq):
+        for si, nb in enumerate(nbs):
+            for I in range(nb):
+                for J in range(I + 1):
+                    idx = h * tri + tri_base[si] + I * (I + 1) // 2 + J
+                    assert flat[idx] == h * 1e6 + si * 1e4 + I * 100 + J, (h, si, I, J)
+                    seen += 1
+    assert seen == flat.size
+
+
+ALL_CHECKS += [check_near_band_is_exactly_the_unforced_ratios_within_the_band,
+               check_triangular_pack_matches_the_layout_formula]

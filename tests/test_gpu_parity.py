@@ -100,8 +100,16 @@ def test_whole_path_matches_oracle():
     ref = O.prefill(q64, k64, v64, data["cu_seqlens"], w.block, 0.1)
     n_near = PT.compare_csr(out["row_ptr"].cpu().numpy(), out["col_idx"].cpu().numpy(),
                             ref["row_ptr"], ref["col_idx"], ref["nears"], w.hq)
-    if n_near == 0:  # same mask -> same attention
+    if n_near == 0:  # same mask: the whole path's own attention output must match
         PT.compare_attention(out["o"], out["lse"], ref["o"], ref["lse"], w.dtype)
+    # always: the attention stage on the oracle's mask
+    pf = out["problem"]
+    ws = fpx.workspace(pf, -1)
+    rp_d = torch.from_numpy(ref["row_ptr"].astype(np.int32)).cuda()
+    ci_d = torch.from_numpy(ref["col_idx"].astype(np.int32)).cuda()
+    o, lse = fpx.sparse_prefill(pf, dev["q"], dev["k"], dev["v"], rp_d, ci_d, ws)
+    assert fpx.status(ws) == 0
+    PT.compare_attention(o, lse, ref["o"], ref["lse"], w.dtype)
 
 
 def test_deterministic():
@@ -121,12 +129,20 @@ def test_device_side_errors_are_recorded():
     pf = PT.gpu_problem(dev, w.block)
     ws = fpx.workspace(pf, -1)
     scores = fpx.block_scores(pf, dev["q"], dev["k"], ws)
-    # col_idx capacity too small: nothing is written, FPX_ERR_CAPACITY recorded
-    col = torch.full((5,), -7, dtype=torch.int32, device="cuda")
-    rp, _, nnz = fpx.select(pf, scores, 0.0, ws, col_idx=col, capacity=5)
+    # col_idx capacity too small: nothing is written, row_ptr is an empty CSR, FPX_ERR_CAPACITY
+    # recorded, nnz reports the count needed.  The capacity is a 5-entry slice of a larger
+    # sentinel-filled buffer, so a write past the slice would show.
+    big = torch.full((64,), -7, dtype=torch.int32, device="cuda")
+    rp, _, nnz = fpx.select(pf, scores, 0.0, ws, col_idx=big, capacity=5)
     assert fpx.status(ws) == -4
-    assert torch.all(col == -7)
+    assert torch.all(big == -7)
+    assert torch.all(rp == 0)
     assert int(nnz.item()) == w.hq * pf.tri
+    # the empty CSR is safe to attend: every row has no key (O = 0, LSE = -inf), nothing read
+    o, lse = fpx.sparse_prefill(pf, dev["q"], dev["k"], dev["v"], rp, big, ws)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+    assert torch.all(big == -7)
     # an index beyond the row's diagonal block: skipped and FPX_ERR_DEVICE_INPUT recorded
     fpx.clear_status(ws)
     rp, ci, _ = fpx.select(pf, scores, 0.0, ws)

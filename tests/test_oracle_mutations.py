@@ -30,6 +30,13 @@ MUTATIONS = {
                                 "    for kp in keeps:\n        for h in range(hq):"),
     "attn_scale_dropped": ("logits = sc * (qt @ kt.T)", "logits = (qt @ kt.T)"),
     "no_renormalise": ("o = (e @ vt) / np.where(ssum > 0, ssum, 1.0)", "o = (e @ vt)"),
+    "near_band_x10": ("NEAR_REL = 1e-3", "NEAR_REL = 1e-2"),
+    "near_band_on_score_difference": ("(np.abs(ratio - alpha) <= NEAR_REL * alpha)",
+                                      "(np.abs((s - m) - alpha) <= NEAR_REL * alpha)"),
+    "near_band_includes_forced": ("near = causal & ~forced & (", "near = causal & ("),
+    "tri_pack_upper_triangle": ("parts.append(s[:, idx[0], idx[1]])",
+                                "parts.append(s[:, idx[1], idx[0]])"),
+    "tri_pack_column_major": ("idx = np.tril_indices(nb)", "idx = np.triu_indices(nb)[::-1]"),
 }
 
 

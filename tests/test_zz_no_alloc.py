@@ -51,3 +51,40 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     a = 0x100000
     rc = lib.fpx_select_noalloc(ctypes.byref(p), a, 0.1, 1, 1, a, a, 10, a, None)
     assert rc == -4  # FPX_ERR_CAPACITY, nothing launched
+
+
+def test_noalloc_reports_overflow_and_bad_cu_seqlens_through_its_outputs():
+    # Both conditions depend on the per-call reset of the status held in the shared scratch: a
+    # normal call after each must again equal fpx_select.
+    w = WORKLOADS["llama8b_bf16_n8192"].with_(seqlens=(300, 0, 129, 640, 1, 128), hq=4, hkv=1,
+                                              q_gain=20.0)
+    dev = PT.to_device(generate(w))
+    pf = PT.gpu_problem(dev, w.block)
+    ws = fpx.workspace(pf, -1)
+    scores = fpx.block_scores(pf, dev["q"], dev["k"], ws)
+    rp_ref, ci_ref, n_ref = fpx.select(pf, scores, 0.1, ws)
+    torch.cuda.synchronize()
+    n = int(n_ref.item())
+
+    def normal_call_matches():
+        rp, ci, nn = fpx.select_noalloc(pf, scores, 0.1)
+        torch.cuda.synchronize()
+        assert torch.equal(rp, rp_ref) and torch.equal(nn, n_ref)
+        assert torch.equal(ci[:n], ci_ref[:n])
+
+    # (1) capacity 5 inside a sentinel-filled buffer: col_idx untouched, empty CSR, full count
+    big = torch.full((64,), -7, dtype=torch.int32, device="cuda")
+    rp, _, nn = fpx.select_noalloc(pf, scores, 0.1, col_idx=big, capacity=5)
+    torch.cuda.synchronize()
+    assert torch.all(big == -7)
+    assert torch.all(rp == 0)
+    assert int(nn.item()) == n
+    normal_call_matches()
+    # (2) device cu_seqlens that disagree with the host mirror: empty CSR, nnz 0
+    cu_good = pf.cu_d.clone()
+    pf.cu_d[2] += 1
+    rp, _, nn = fpx.select_noalloc(pf, scores, 0.1)
+    torch.cuda.synchronize()
+    assert torch.all(rp == 0) and int(nn.item()) == 0
+    pf.cu_d.copy_(cu_good)
+    normal_call_matches()
