@@ -51,20 +51,48 @@ def probe_attention(q, k, start: int, n: int, pos: np.ndarray, scale: float, g: 
     return a
 
 
-def vertical_slash(a: np.ndarray, pos: np.ndarray, alpha_v: float, alpha_s: float
-                   ) -> Tuple[List[np.ndarray], List[np.ndarray]]:
-    """Per Q head: sorted vertical key tokens and sorted slash offsets of one sequence."""
+def probe_scores(a: np.ndarray, pos: np.ndarray) -> Tuple[List[np.ndarray], List[np.ndarray]]:
+    """Per Q head: v [n], the vertical significance of every key token (max over the probes that
+    see it), and d [n], the slash significance of every offset (max over the probes of the
+    probability that many tokens back)."""
     hq, _, n = a.shape
-    verts, slashes = [], []
+    vs, ds = [], []
     for h in range(hq):
         v = np.zeros(n)
         d = np.zeros(n)
         for p, i in enumerate(pos):
             v[:i + 1] = np.maximum(v[:i + 1], a[h, p, :i + 1])
             d[:i + 1] = np.maximum(d[:i + 1], a[h, p, i::-1])  # offset delta = i - j
-        verts.append(np.arange(n) if alpha_v == 0 else np.nonzero(v >= alpha_v * v.max())[0])
-        slashes.append(np.arange(n) if alpha_s == 0 else np.nonzero(d >= alpha_s * d.max())[0])
+        vs.append(v)
+        ds.append(d)
+    return vs, ds
+
+
+def _select_max_based(x: np.ndarray, alpha: float) -> np.ndarray:
+    if alpha == 0:
+        return np.arange(x.size)
+    if x.size == 0:
+        return np.zeros(0, np.int64)
+    return np.nonzero(x >= alpha * x.max())[0]
+
+
+def vertical_slash(a: np.ndarray, pos: np.ndarray, alpha_v: float, alpha_s: float
+                   ) -> Tuple[List[np.ndarray], List[np.ndarray]]:
+    """Per Q head: sorted vertical key tokens and sorted slash offsets of one sequence."""
+    vs, ds = probe_scores(a, pos)
+    verts = [_select_max_based(v, alpha_v) for v in vs]
+    slashes = [_select_max_based(d, alpha_s) for d in ds]
     return verts, slashes
+
+
+def near_threshold(x: np.ndarray, alpha: float) -> np.ndarray:
+    """Indices whose significance lies within NEAR_REL * alpha * max of the selection threshold
+    alpha * max (alpha > 0): decisions there may flip with rounding and are reported, not
+    failed (the same rule as the block threshold's)."""
+    if alpha == 0 or x.size == 0:
+        return np.zeros(0, np.int64)
+    thr = alpha * x.max()
+    return np.nonzero(np.abs(x - thr) <= O.NEAR_REL * thr)[0]
 
 
 def token_mask(n: int, verts: np.ndarray, slashes: np.ndarray) -> np.ndarray:
@@ -89,6 +117,8 @@ def attention_token_mask(q, k, v, cu_seqlens, masks: List[np.ndarray], scale=Non
     lse = np.full((hq, t_all), -np.inf)
     for s_, L in enumerate(O.seq_layout(cu_seqlens, 1)):
         a, n = L["start"], L["n"]
+        if n == 0:  # an empty sequence has no rows
+            continue
         for h in range(hq):
             qq = np.asarray(q[a:a + n, h], np.float64)
             kk = np.asarray(k[a:a + n, h // g], np.float64)
@@ -103,9 +133,10 @@ def attention_token_mask(q, k, v, cu_seqlens, masks: List[np.ndarray], scale=Non
     return o, lse
 
 
-def discover(q, k, cu_seqlens, n_probe: int, alpha_v: float, alpha_s: float, scale=None
-             ) -> List[Tuple[List[np.ndarray], List[np.ndarray]]]:
-    """Per sequence: (verticals per head, slashes per head)."""
+def discover(q, k, cu_seqlens, n_probe: int, alpha_v: float, alpha_s: float, scale=None,
+             with_near: bool = False):
+    """Per sequence: (verticals per head, slashes per head); with_near: also the near-threshold
+    key tokens and offsets per head, (verts, slashes, near_verts, near_slashes)."""
     hq, d = q.shape[1], q.shape[2]
     g = hq // k.shape[1]
     sc = O.default_scale(d) if scale is None or scale <= 0 else float(scale)
@@ -113,5 +144,47 @@ def discover(q, k, cu_seqlens, n_probe: int, alpha_v: float, alpha_s: float, sca
     for L in O.seq_layout(cu_seqlens, 1):
         pos = probe_positions(L["n"], n_probe)
         a = probe_attention(q, k, L["start"], L["n"], pos, sc, g)
-        out.append(vertical_slash(a, pos, alpha_v, alpha_s))
+        if not with_near:
+            out.append(vertical_slash(a, pos, alpha_v, alpha_s))
+            continue
+        vs, ds = probe_scores(a, pos)
+        out.append(([_select_max_based(v, alpha_v) for v in vs],
+                     [_select_max_based(x, alpha_s) for x in ds],
+                     [near_threshold(v, alpha_v) for v in vs],
+                     [near_threshold(x, alpha_s) for x in ds]))
     return out
+
+
+def attention_token_rows(q, k, v, cu_seqlens, verts, slashes, rows, scale=None):
+    """O [len(rows), D] and LSE [len(rows)] of exact attention for the listed (h, t) pairs (t a
+    global token index) under the vertical / slash token mask: query i of sequence s attends key
+    j <= i iff j is in verts[s][h] or i - j is in slashes[s][h]; a row with no key gets O = 0,
+    LSE = -inf.  The same definition as attention_token_mask, evaluated row by row."""
+    hq, d = q.shape[1], q.shape[2]
+    g = hq // k.shape[1]
+    sc = O.default_scale(d) if scale is None or scale <= 0 else float(scale)
+    lay = O.seq_layout(cu_seqlens, 1)
+    starts = np.array([L["start"] for L in lay])
+    o = np.zeros((len(rows), v.shape[2]))
+    lse = np.full(len(rows), -np.inf)
+    for r, (h, t) in enumerate(rows):
+        s_ = int(np.searchsorted(starts, t, side="right") - 1)
+        while lay[s_]["n"] == 0 or t >= lay[s_]["start"] + lay[s_]["n"]:
+            s_ += 1
+        a, n = lay[s_]["start"], lay[s_]["n"]
+        i = t - a
+        isv = np.zeros(n, bool)
+        isv[np.asarray(verts[s_][h], np.int64)] = True
+        iss = np.zeros(n, bool)
+        iss[np.asarray(slashes[s_][h], np.int64)] = True
+        j = np.arange(i + 1)
+        keys = j[isv[j] | iss[i - j]]
+        if keys.size == 0:
+            continue
+        logits = sc * (np.asarray(k[a + keys, h // g], np.float64) @
+                       np.asarray(q[t, h], np.float64))
+        m = logits.max()
+        e = np.exp(logits - m)
+        lse[r] = m + np.log(e.sum())
+        o[r] = (e / e.sum()) @ np.asarray(v[a + keys, h // g], np.float64)
+    return o, lse

@@ -37,7 +37,11 @@ MUTATIONS = {
         "probe_not_causal": ("logits = scale * (kk[:i + 1] @", "logits = scale * (kk[:i + 2] @"),
         "attn_scale_dropped": ("logits = np.where(masks[s_][h], sc * (qq @ kk.T), -np.inf)",
                                "logits = np.where(masks[s_][h], (qq @ kk.T), -np.inf)"),
-        "threshold_inverted": ("np.nonzero(v >= alpha_v * v.max())", "np.nonzero(v <= alpha_v * v.max())"),
+        "threshold_inverted": ("np.nonzero(x >= alpha * x.max())", "np.nonzero(x <= alpha * x.max())"),
+        "near_band_x10": ("np.abs(x - thr) <= O.NEAR_REL * thr", "np.abs(x - thr) <= 10 * O.NEAR_REL * thr"),
+        "near_band_absolute": ("np.abs(x - thr) <= O.NEAR_REL * thr", "np.abs(x - thr) <= O.NEAR_REL"),
+        "token_rows_offset_sign": ("keys = j[isv[j] | iss[i - j]]", "keys = j[isv[j] | iss[j]]"),
+        "token_rows_not_causal": ("j = np.arange(i + 1)", "j = np.arange(min(i + 2, n))"),
     }),
 }
 

@@ -91,7 +91,39 @@ def check_aggregation_over_probes_is_the_max(PO=PO):
     assert slashes[0].tolist() == [1]
 
 
-ALL_CHECKS = [check_probe_positions_are_uniform_and_end_at_the_last_token,
+def check_near_threshold_band(PO=PO):
+    # significances placed at known distances from alpha * max: inside the 1e-3 relative band
+    # (+-5e-4, -9e-4 of the threshold) and outside it (+-2e-3)
+    for alpha in (0.05, 0.3, 0.9):
+        x = np.array([1.0, alpha * (1 + 5e-4), alpha * (1 - 9e-4), alpha * (1 + 2e-3),
+                      alpha * (1 - 2e-3), alpha * (1 - 5e-4), 0.0]) * 0.37
+        assert PO.near_threshold(x, alpha).tolist() == [1, 2, 5]
+        assert PO._select_max_based(x, alpha).tolist() == [0, 1, 3]
+    assert PO.near_threshold(x, 0.0).size == 0
+    assert PO.near_threshold(np.zeros(0), 0.5).size == 0
+
+
+def check_token_rows_equal_full_token_mask_attention(PO=PO):
+    rng = np.random.default_rng(4)
+    t, hq, hkv, d = 50, 2, 1, 8
+    q, k, v = (rng.standard_normal((t, h, d)) for h in (hq, hkv, hkv))
+    cu = [0, 21, 21, 50]
+    verts = [[np.array([0, 5]), np.array([3])], [[], []], [np.array([1, 20]), np.array([])]]
+    slashes = [[np.array([0, 2]), np.array([4])], [[], []], [np.array([0]), np.array([1, 7])]]
+    masks = [[PO.token_mask(n, np.asarray(vs[h], int), np.asarray(ss[h], int)) for h in range(hq)]
+             for n, vs, ss in zip([21, 0, 29], verts, slashes)]
+    o, lse = PO.attention_token_mask(q, k, v, cu, masks)
+    # includes rows whose next key is a vertical (0, 4) and (1, 2): a non-causal row would see it
+    rows = [(0, 0), (1, 0), (1, 3), (0, 20), (1, 21), (0, 49), (1, 30), (0, 25), (0, 4), (1, 2)]
+    o_r, lse_r = PO.attention_token_rows(q, k, v, cu, verts, slashes, rows)
+    for n_, (h, t_) in enumerate(rows):
+        assert lse_r[n_] == lse[h, t_] or abs(lse_r[n_] - lse[h, t_]) < 1e-12
+        assert np.abs(o_r[n_] - o[t_, h]).max() < 1e-12
+    assert np.isneginf(lse_r[1]) and not o_r[1].any()  # head 1, token 0: no key at all
+
+
+ALL_CHECKS = [check_near_threshold_band, check_token_rows_equal_full_token_mask_attention,
+              check_probe_positions_are_uniform_and_end_at_the_last_token,
               check_alpha_zero_is_dense_causal_attention, check_planted_vertical_and_slash_are_found,
               check_token_masked_attention_matches_brute_force, check_threshold_edges,
               check_aggregation_over_probes_is_the_max]
@@ -119,3 +151,11 @@ def test_threshold_edges():
 
 def test_aggregation_over_probes_is_the_max():
     check_aggregation_over_probes_is_the_max()
+
+
+def test_near_threshold_band():
+    check_near_threshold_band()
+
+
+def test_token_rows_equal_full_token_mask_attention():
+    check_token_rows_equal_full_token_mask_attention()
