@@ -265,52 +265,167 @@ def extras(fpx, w, pf, dev, cu, ws, scores, row_ptr, col_idx, device, reps=3):
     return out
 
 
+class Prefill:
+    """One workload resident on the device with every buffer of the path allocated once; step()
+    enqueues the whole hot path (fpx_block_scores -> fpx_select -> fpx_sparse_prefill) on the
+    current stream and, when asked, records CUDA events around the search and the attention."""
+
+    def __init__(self, fpx, w, data, device, host_copies=False):
+        self.fpx, self.w, self.device = fpx, w, device
+        self.cu = data["cu_seqlens"]
+        if host_copies:
+            self.host = {k: data[k].contiguous().pin_memory() for k in ("q", "k", "v")}
+            self.dev = {k: self.host[k].to(device, non_blocking=True) for k in self.host}
+        else:
+            self.host = None
+            self.dev = {k: data[k].to(device) for k in ("q", "k", "v")}
+        for k in ("q_scale", "k_scale", "v_scale"):
+            self.dev[k] = data[k].to(device) if data[k] is not None else None
+        torch.cuda.synchronize(device)
+        d = self.dev
+        self.stream = torch.cuda.current_stream(device)
+        self.pf = fpx.problem(d["q"], d["k"], w.block, self.cu, 0.0, d["q_scale"], d["k_scale"],
+                              d["v_scale"])
+        pf = self.pf
+        self.ws = fpx.workspace(pf, -1, device)
+        self.scores = torch.empty(w.hq * pf.tri, dtype=torch.float32, device=device)
+        self.row_ptr = torch.empty(pf.rows + 1, dtype=torch.int32, device=device)
+        self.col_idx = torch.empty(max(1, w.hq * pf.tri), dtype=torch.int32, device=device)
+        self.nnz = torch.empty(1, dtype=torch.int64, device=device)
+        self.o = torch.empty(d["q"].shape, dtype=torch.float32 if w.dtype == "f32"
+                             else torch.bfloat16, device=device)
+        self.lse = torch.empty((w.hq, w.total_tokens), dtype=torch.float32, device=device)
+
+    def step(self, timing=None):
+        fpx, w, d = self.fpx, self.w, self.dev
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(self.stream)
+        fpx.block_scores(self.pf, d["q"], d["k"], self.ws, scores=self.scores)
+        fpx.select(self.pf, self.scores, w.alpha, self.ws, w.sink_blocks, w.window_blocks,
+                   row_ptr=self.row_ptr, col_idx=self.col_idx, nnz=self.nnz)
+        e1.record(self.stream)
+        fpx.sparse_prefill(self.pf, d["q"], d["k"], d["v"], self.row_ptr, self.col_idx, self.ws,
+                           o=self.o, lse=self.lse)
+        e2.record(self.stream)
+        if timing is not None:
+            timing.append((e0, e1, e2))
+
+    def check_status(self, when: str):
+        st = self.fpx.status(self.ws)
+        if st != 0:
+            raise RuntimeError(f"device status {st} {when}")
+
+    def metrics(self, search_ms, attn_ms, n_kept):
+        """The per-workload figures of the metric, from per-step CUDA-event times."""
+        w = self.w
+        pk, pk_kind = peaks()
+        peak_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        if w.dtype == "e4m3":
+            peak_tf *= 2.0  # fp8 dense is twice bf16 (nominal ratio)
+        tri = pairs(w)
+        attn = statistics.mean(attn_ms)
+        srch = statistics.mean(search_ms)
+        exec_tf = 4.0 * w.block * w.block * w.d * n_kept / (attn * 1e-3) / 1e12
+        dq, dk = self.dev["q"], self.dev["k"]
+        # algorithmic bytes of the search: Q and K read once, the pooled scores written once, the
+        # CSR written (the select pass's read-back of the scores is reported apart, not counted)
+        sbytes = (dq.numel() * dq.element_size() + dk.numel() * dk.element_size() +
+                  4 * w.hq * tri + 4 * (self.pf.rows + 1) + 4 * n_kept)
+        gbs = sbytes / (srch * 1e-3) / 1e9
+        flops = dense_flops(w)
+        return {
+            "attn_ms": round(attn, 4), "search_ms": round(srch, 4),
+            "density": round(n_kept / (w.hq * tri), 6), "nnz": n_kept,
+            "attn_dense_equiv_tflops": round(flops / (attn * 1e-3) / 1e12, 3),
+            "step_dense_equiv_tflops": round(flops / ((attn + srch) * 1e-3) / 1e12, 3),
+            "attn_executed_tflops": round(exec_tf, 2),
+            "attn_executed_frac": round(exec_tf / peak_tf, 4),
+            "attn_peak": {"tflops": peak_tf, "kind": f"{pk_kind} bf16 sustained" +
+                          (" x2 (fp8, nominal ratio)" if w.dtype == "e4m3" else "")},
+            "search_bytes": sbytes, "search_gbs": round(gbs, 1),
+            "search_hbm_frac": round(gbs / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), 4),
+        }
+
+    def measure(self, steps, warmup):
+        """warmup untimed steps, then `steps` steps with per-step events; the figures above."""
+        for _ in range(warmup):
+            self.step()
+        self.check_status("after warm-up")
+        n_kept = int(self.nnz.item())
+        torch.cuda.synchronize(self.device)
+        timing = []
+        with ClockSampler(self.device.index if self.device.index is not None else 0) as clk:
+            for _ in range(steps):
+                self.step(timing)
+            torch.cuda.synchronize(self.device)
+        self.check_status("after the timed steps")
+        res = self.metrics([a.elapsed_time(b) for a, b, c in timing],
+                           [b.elapsed_time(c) for a, b, c in timing], n_kept)
+        res["clocks"] = clk.summary()
+        return res
+
+
+def sub_records(fpx, args, device, sdpa_ms_128k):
+    """The other configurations of the metric, timed by the same code after the headline's timed
+    region (each: 3 warm-up steps, then args.sub_steps timed steps; every workload's Q + K + V is
+    larger than L2, so no flush is needed between steps).
+    * sparse: the 131072-token layer with Q multiplied by q_gain (a labelled supplementary knob
+      that widens the pooled-score spread as trained models' logits do): alpha = 0.1 then keeps
+      about 50 %, 20 % and 5 % of the causal blocks; speed-up over the same run's dense SDPA;
+    * llama8b_bf16_n32768 at alpha 0, 0.05, 0.1, 0.2; llama8b_e4m3_n131072; varlen8_bf16_t264192.
+    """
+    out = {"sparse": [], "configs": []}
+    steps = args.sub_steps
+    base = WORKLOADS["llama8b_bf16_n131072"]
+    # one fp32 draw; Q for each gain is bf16(q_gain * q_fp32), exactly what the generator
+    # produces for that gain
+    f32 = generate(base.with_(dtype="f32"), workers=default_workers())
+    for gain in (290.0, 340.0, 415.0):
+        w = base.with_(q_gain=gain)
+        data = dict(f32, q=(f32["q"] * np.float32(gain)).to(torch.bfloat16),
+                    k=f32["k"].to(torch.bfloat16), v=f32["v"].to(torch.bfloat16))
+        run = Prefill(fpx, w, data, device)
+        r = run.measure(steps, 3)
+        del run, data
+        torch.cuda.empty_cache()
+        r = {"workload": w.name, "q_gain": gain, "alpha": w.alpha, **r}
+        if sdpa_ms_128k:
+            r["speedup_vs_sdpa_dense"] = round(sdpa_ms_128k / r["attn_ms"], 3)
+        out["sparse"].append(r)
+    del f32
+    for name, alphas in (("llama8b_bf16_n32768", (0.0, 0.05, 0.1, 0.2)),
+                         ("llama8b_e4m3_n131072", (None,)), ("varlen8_bf16_t264192", (None,))):
+        w0 = WORKLOADS[name]
+        data = generate(w0, workers=default_workers())
+        for a in alphas:
+            w = w0 if a is None else w0.with_(alpha=a)
+            run = Prefill(fpx, w, data, device)
+            r = run.measure(steps, 3)
+            del run
+            torch.cuda.empty_cache()
+            out["configs"].append({"workload": w.name, "alpha": w.alpha, **r})
+        del data
+    return out
+
+
 def run_ours(args, rank, world, device):
     import dynamic_block_sparse_pooled_b200 as fpx
 
     w = WORKLOADS[args.workload]
     if args.alpha is not None:
         w = w.with_(alpha=args.alpha)
+    if args.q_gain is not None:
+        w = w.with_(q_gain=args.q_gain)
     data = generate(w, workers=default_workers())
-    cu = data["cu_seqlens"]
-    host = {k: data[k].contiguous().pin_memory() for k in ("q", "k", "v")}
-    dev = {k: host[k].to(device, non_blocking=True) for k in host}
-    for k in ("q_scale", "k_scale", "v_scale"):
-        dev[k] = data[k].to(device) if data[k] is not None else None
-    torch.cuda.synchronize(device)
-
-    stream = torch.cuda.current_stream(device)
-    pf = fpx.problem(dev["q"], dev["k"], w.block, cu, 0.0, dev["q_scale"], dev["k_scale"],
-                     dev["v_scale"])
-    ws = fpx.workspace(pf, -1, device)
-    scores = torch.empty(w.hq * pf.tri, dtype=torch.float32, device=device)
-    row_ptr = torch.empty(pf.rows + 1, dtype=torch.int32, device=device)
-    col_idx = torch.empty(max(1, w.hq * pf.tri), dtype=torch.int32, device=device)
-    nnz = torch.empty(1, dtype=torch.int64, device=device)
-    o = torch.empty(dev["q"].shape, dtype=torch.bfloat16 if w.dtype != "f32" else torch.float32,
-                    device=device)
-    lse = torch.empty((w.hq, w.total_tokens), dtype=torch.float32, device=device)
-
+    run = Prefill(fpx, w, data, device, host_copies=True)
+    stream = run.stream
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def step(timing=None):
-        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
-        e0.record(stream)
-        fpx.block_scores(pf, dev["q"], dev["k"], ws, scores=scores)
-        fpx.select(pf, scores, w.alpha, ws, w.sink_blocks, w.window_blocks, row_ptr=row_ptr,
-                   col_idx=col_idx, nnz=nnz)
-        e1.record(stream)
-        fpx.sparse_prefill(pf, dev["q"], dev["k"], dev["v"], row_ptr, col_idx, ws, o=o, lse=lse)
-        e2.record(stream)
-        if timing is not None:
-            timing.append((e0, e1, e2))
-
     for _ in range(args.warmup):
-        step()
-    st = fpx.status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st} after warm-up")
-    n_kept = int(nnz.item())
+        run.step()
+    run.check_status("after warm-up")
+    n_kept = int(run.nnz.item())
 
     if world > 1:
         torch.distributed.barrier()
@@ -320,7 +435,7 @@ def run_ours(args, rank, world, device):
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t_start.record(stream)
         for _ in range(args.steps):
-            step(timing)
+            run.step(timing)
         t_end.record(stream)
         torch.cuda.synchronize(device)
     if world > 1:
@@ -328,13 +443,12 @@ def run_ours(args, rank, world, device):
     total_ms = t_start.elapsed_time(t_end)
     search_ms = [a.elapsed_time(b) for a, b, c in timing]
     attn_ms = [b.elapsed_time(c) for a, b, c in timing]
-    st = fpx.status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st} after the timed steps")
+    run.check_status("after the timed steps")
 
     # end to end through the public API: pinned host Q/K/V -> device, whole path, O + LSE -> host
-    host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    host_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    host, dev = run.host, run.dev
+    host_o = torch.empty(run.o.shape, dtype=run.o.dtype, pin_memory=True)
+    host_lse = torch.empty(run.lse.shape, dtype=run.lse.dtype, pin_memory=True)
     e2e_steps = max(1, min(args.steps, 3))
     torch.cuda.synchronize(device)
     a, b = ev(), ev()
@@ -342,9 +456,9 @@ def run_ours(args, rank, world, device):
     for _ in range(e2e_steps):
         for k in ("q", "k", "v"):
             dev[k].copy_(host[k], non_blocking=True)
-        step()
-        host_o.copy_(o, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
+        run.step()
+        host_o.copy_(run.o, non_blocking=True)
+        host_lse.copy_(run.lse, non_blocking=True)
     b.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = a.elapsed_time(b) / e2e_steps
@@ -354,20 +468,9 @@ def run_ours(args, rank, world, device):
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device)
     ms_step = total_ms / args.steps
     flops = dense_flops(w)
-    tri = pairs(w)
-    density = n_kept / (w.hq * tri)
-    attn_avg = statistics.mean(attn_ms)
-    exec_flops = 4.0 * w.block * w.block * w.d * n_kept
-    pk, pk_kind = peaks()
-    peak_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    if w.dtype == "e4m3":
-        peak_tf *= 2.0  # fp8 dense is twice bf16 (nominal ratio)
-    achieved = exec_flops / (attn_avg * 1e-3) / 1e12
-    # algorithmic bytes of the search: Q and K read once, the pooled scores written once, the CSR
-    # written (the select pass's read-back of the scores is reported apart, not counted)
-    search_bytes = (dev["q"].numel() * dev["q"].element_size() +
-                    dev["k"].numel() * dev["k"].element_size() +
-                    4 * w.hq * tri + 4 * (pf.rows + 1) + 4 * n_kept)
+    m = run.metrics(search_ms, attn_ms, n_kept)
+    achieved = m["attn_executed_tflops"]
+    peak_tf = m["attn_peak"]["tflops"]
     res = {
         "metric": METRIC,
         "value": round(aggregate_value(flops, world, ms_step), 3),
@@ -377,18 +480,15 @@ def run_ours(args, rank, world, device):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded generator: RoPE + sink + verticals + slash)",
         "config": config_of(w, world),
-        "attn_ms": round(attn_avg, 4),
-        "search_ms": round(statistics.mean(search_ms), 4),
-        "attn_dense_equiv_tflops": round(flops / (attn_avg * 1e-3) / 1e12, 3),
-        "density": round(density, 6), "nnz": n_kept,
-        "search_bytes": search_bytes, "search_scores_readback_bytes": 4 * w.hq * tri,
-        "search_gbs": round(search_bytes / (statistics.mean(search_ms) * 1e-3) / 1e9, 1),
-        "search_hbm_frac": round(search_bytes / (statistics.mean(search_ms) * 1e-3) / 1e9
-                                 / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), 4),
-        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(achieved, 2),
+        "attn_ms": m["attn_ms"], "search_ms": m["search_ms"],
+        "attn_dense_equiv_tflops": m["attn_dense_equiv_tflops"],
+        "density": m["density"], "nnz": n_kept,
+        "search_bytes": m["search_bytes"], "search_scores_readback_bytes": 4 * w.hq * pairs(w),
+        "search_gbs": m["search_gbs"], "search_hbm_frac": m["search_hbm_frac"],
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
-                     "peak_kind": f"{pk_kind} bf16 sustained" + (" x2 (fp8)" if w.dtype == "e4m3" else ""),
-                     "traffic": attn_traffic(w.name),
+                     "peak_kind": m["attn_peak"]["kind"],
+                     "traffic": attn_traffic(w.name) if w.q_gain == 1.0 else None,
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "per_launch": "executed FLOP = 4*B^2*D*nnz (every kept 128x128 tile)"},
         "e2e": {"value": round(aggregate_value(flops, world, e2e_ms), 3),
@@ -396,11 +496,18 @@ def run_ours(args, rank, world, device):
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
-        "sdpa_baseline": sdpa_baseline(w, dev, cu, device) if not args.no_sdpa else None,
-        "extras": extras(fpx, w, pf, dev, cu, ws, scores, row_ptr, col_idx, device)
-        if not args.no_sdpa else None,
         "clocks": clk.summary(),
     }
+    if not args.no_sdpa:
+        res["sdpa_baseline"] = sdpa_baseline(w, dev, run.cu, device)
+        res["extras"] = extras(fpx, w, run.pf, dev, run.cu, run.ws, run.scores, run.row_ptr,
+                               run.col_idx, device)
+    del run, host, dev
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_sub and args.workload == DEFAULT_WORKLOAD and \
+            args.alpha is None and args.q_gain is None:
+        sd = res.get("sdpa_baseline") or {}
+        res["sub_records"] = sub_records(fpx, args, device, sd.get("ms"))
     return res, w, data
 
 
@@ -496,6 +603,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sdpa", action="store_true",
                     help="skip the PyTorch SDPA baseline and the paged / rescue timings")
+    ap.add_argument("--q-gain", type=float, default=None,
+                    help="multiply Q by this gain (the labelled sparse-regime knob)")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="skip the sub-records (sparse sweep, 32K, e4m3, varlen)")
+    ap.add_argument("--sub-steps", type=int, default=5, help="timed steps per sub-record")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

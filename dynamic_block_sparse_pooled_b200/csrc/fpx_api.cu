@@ -112,8 +112,8 @@ size_t scratch_bytes(const fpx_problem* p, const Sizes& s, int which) {
       return align_up(sizeof(float) * R, 256) + align_up(sizeof(int32_t) * R, 256) +
              align_up(sizeof(int64_t) * (R / 8 + 1), 256) + 256 +
              align_up(sizeof(uint32_t) * R * mask_words(s), 256);
-    case 2:  // tile schedule
-      return align_up(sizeof(int32_t) * R, 256);
+    case 2:  // tile schedule + the persistent kernel's work-queue head
+      return align_up(sizeof(int32_t) * R, 256) + 256;
     default:
       return 0;
   }
@@ -121,6 +121,51 @@ size_t scratch_bytes(const fpx_problem* p, const Sizes& s, int which) {
 
 size_t ws_bytes_for(const fpx_problem* p, const Sizes& s, int which) {
   return scratch_offset(p->num_seqs) + scratch_bytes(p, s, which);
+}
+
+// ---- query-probe vertical / slash path ---------------------------------------------------
+constexpr int kProbeChunkBlocks = 8;  // key blocks of 128 per probe CTA
+
+int pattern_words(const fpx_problem* p) { return (p->total_tokens + 31) / 32; }
+
+int64_t probe_chunks(const fpx_problem* p) {
+  // sum over sequences of ceil(nb_s / chunk) with nb_s counted in 128-key blocks
+  int64_t c = 0;
+  for (int i = 0; i < p->num_seqs; ++i) {
+    const int64_t n = p->cu_seqlens_h ? static_cast<int64_t>(p->cu_seqlens_h[i + 1]) -
+                                            p->cu_seqlens_h[i]
+                                      : p->total_tokens;
+    const int64_t nb = (n + 127) / 128;
+    c += (nb + kProbeChunkBlocks - 1) / kProbeChunkBlocks;
+  }
+  return c;
+}
+
+struct ProbeLayout {
+  size_t chunk_base, partial, bound, end;  // byte offsets inside the workspace
+};
+
+ProbeLayout probe_layout(const fpx_problem* p, int n_probe) {
+  const int tiles = (p->hq / p->hkv * n_probe + 127) / 128;
+  ProbeLayout L;
+  L.chunk_base = scratch_offset(p->num_seqs);
+  L.partial = L.chunk_base + align_up(sizeof(int32_t) * (p->num_seqs + 1), 256);
+  L.bound = L.partial + align_up(sizeof(float) * 2 * static_cast<size_t>(probe_chunks(p)) *
+                                     p->hkv * tiles * 128, 256);
+  L.end = L.bound + align_up(sizeof(float) * 2 * static_cast<size_t>(p->num_seqs) * p->hq *
+                                 n_probe, 256);
+  return L;
+}
+
+// vs_select: the select stage's scratch followed by the two per-(head, block) flag arrays
+size_t vs_select_bytes(const fpx_problem* p, const Sizes& s) {
+  return ws_bytes_for(p, s, 1) + 2 * align_up(static_cast<size_t>(s.nb) * p->hq, 256);
+}
+
+fpx_status check_probe_args(const fpx_problem* p, int n_probe) {
+  if (n_probe < 1 || static_cast<int64_t>(p->hq / p->hkv) * n_probe > 512)
+    return FPX_ERR_UNSUPPORTED;
+  return FPX_OK;
 }
 
 fpx_status check_ws(const fpx_problem* p, const Sizes& s, int which, void* ws, size_t ws_bytes) {
@@ -325,7 +370,8 @@ static fpx_status sparse_prefill_impl(const fpx_problem* p, const void* q, const
                                       const void* v, const fpx_paged_kv* kv,
                                       const int32_t* row_ptr, const int32_t* col_idx, void* o,
                                       float* lse, void* ws, size_t ws_bytes,
-                                      fpx_stream_t stream) {
+                                      fpx_stream_t stream, const uint32_t* vbits = nullptr,
+                                      const uint32_t* sbits = nullptr) {
   Sizes sz;
   fpx_status rc = check_problem(p, &sz);
   if (rc != FPX_OK) return rc;
@@ -344,13 +390,18 @@ static fpx_status sparse_prefill_impl(const fpx_problem* p, const void* q, const
   const SeqTables t = seq_tables_at(ws, p->num_seqs);
   char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
   int32_t* order = reinterpret_cast<int32_t*>(scratch);
+  int* queue_head = reinterpret_cast<int*>(
+      scratch + align_up(sizeof(int32_t) * static_cast<size_t>(sz.nb) * p->hq, 256));
   if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
   if (sz.nb == 0) return FPX_OK;
   const bool tc = attn_tc_supported(d, p->dtype);
-  if (launch_order(d, t, order, tc, s) != cudaSuccess) return FPX_ERR_CUDA;
+  if (launch_order(d, static_cast<int>(sz.nb_max), t, row_ptr, order, queue_head, tc, s) !=
+      cudaSuccess)
+    return FPX_ERR_CUDA;
   if (tc) {
     bool encode_failed = false;
-    cudaError_t e = launch_attn_tc(d, p->dtype, q, k, v, row_ptr, col_idx, o, lse, t, order, st, s,
+    cudaError_t e = launch_attn_tc(d, p->dtype, q, k, v, row_ptr, col_idx, o, lse, t, order,
+                                   queue_head, vbits, sbits, pattern_words(p), st, s,
                                    &encode_failed);
     if (encode_failed) return FPX_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FPX_OK : FPX_ERR_CUDA;
@@ -364,6 +415,110 @@ fpx_status fpx_sparse_prefill(const fpx_problem* p, const void* q, const void* k
                               const int32_t* row_ptr, const int32_t* col_idx, void* o,
                               float* lse, void* ws, size_t ws_bytes, fpx_stream_t stream) {
   return sparse_prefill_impl(p, q, k, v, nullptr, row_ptr, col_idx, o, lse, ws, ws_bytes, stream);
+}
+
+size_t fpx_pattern_words(const fpx_problem* p) {
+  Sizes s;
+  return check_problem(p, &s) == FPX_OK ? static_cast<size_t>(pattern_words(p)) : 0;
+}
+
+size_t fpx_vs_workspace_bytes(const fpx_problem* p, int32_t n_probe) {
+  Sizes s;
+  if (check_problem(p, &s) != FPX_OK || check_probe_args(p, n_probe) != FPX_OK) return 0;
+  size_t m = probe_layout(p, n_probe).end;
+  m = std::max(m, vs_select_bytes(p, s));
+  return std::max(m, ws_bytes_for(p, s, 2));
+}
+
+fpx_status fpx_probe_patterns(const fpx_problem* p, const void* q, const void* k,
+                              int32_t n_probe, float alpha_v, float alpha_s, uint32_t* vert_bits,
+                              uint32_t* slash_bits, void* ws, size_t ws_bytes,
+                              fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if ((rc = check_probe_args(p, n_probe)) != FPX_OK) return rc;
+  ProblemDesc d = make_desc(p, sz);
+  if (!attn_tc_supported(d, p->dtype)) return FPX_ERR_UNSUPPORTED;
+  if (std::isnan(alpha_v) || std::isnan(alpha_s) || alpha_v < 0.f || alpha_s < 0.f)
+    return FPX_ERR_INVALID_ARG;
+  if (!ws) return FPX_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return FPX_ERR_ALIGNMENT;
+  const ProbeLayout L = probe_layout(p, n_probe);
+  if (ws_bytes < L.end) return FPX_ERR_CAPACITY;
+  if (p->total_tokens > 0 && (!q || !k || !vert_bits || !slash_bits)) return FPX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(vert_bits, 4) || !aligned(slash_bits, 4))
+    return FPX_ERR_ALIGNMENT;
+  if (probe_chunks(p) >= INT32_MAX) return FPX_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  StatusBlock* st = static_cast<StatusBlock*>(ws);
+  const SeqTables t = seq_tables_at(ws, p->num_seqs);
+  char* base = static_cast<char*>(ws);
+  if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
+  bool encode_failed = false;
+  cudaError_t e = launch_probe(
+      d, p->dtype, q, k, n_probe, alpha_v, alpha_s, kProbeChunkBlocks,
+      static_cast<int>(probe_chunks(p)), t, reinterpret_cast<int32_t*>(base + L.chunk_base),
+      reinterpret_cast<float2*>(base + L.partial), reinterpret_cast<float2*>(base + L.bound),
+      vert_bits, slash_bits, pattern_words(p), st, s, &encode_failed);
+  if (encode_failed) return FPX_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FPX_OK : FPX_ERR_CUDA;
+}
+
+fpx_status fpx_vs_select(const fpx_problem* p, const uint32_t* vert_bits,
+                         const uint32_t* slash_bits, int32_t* row_ptr, int32_t* col_idx,
+                         int64_t col_capacity, int64_t* nnz_d, void* ws, size_t ws_bytes,
+                         fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  const ProblemDesc d = make_desc(p, sz);
+  if (!attn_tc_supported(d, p->dtype)) return FPX_ERR_UNSUPPORTED;
+  if (!ws) return FPX_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return FPX_ERR_ALIGNMENT;
+  if (ws_bytes < vs_select_bytes(p, sz)) return FPX_ERR_CAPACITY;
+  if (col_capacity < 0 || !row_ptr) return FPX_ERR_INVALID_ARG;
+  if (p->total_tokens > 0 && (!vert_bits || !slash_bits || (!col_idx && col_capacity > 0)))
+    return FPX_ERR_INVALID_ARG;
+  if (!aligned(vert_bits, 4) || !aligned(slash_bits, 4) || !aligned(row_ptr, 4) ||
+      !aligned(col_idx, 4) || !aligned(nnz_d, 8))
+    return FPX_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  StatusBlock* st = static_cast<StatusBlock*>(ws);
+  const SeqTables t = seq_tables_at(ws, p->num_seqs);
+  const size_t R = static_cast<size_t>(sz.nb) * p->hq;
+  char* scratch = static_cast<char*>(ws) + scratch_offset(p->num_seqs);
+  int32_t* counts = reinterpret_cast<int32_t*>(scratch + align_up(sizeof(float) * R, 256));
+  int64_t* cta_tot = reinterpret_cast<int64_t*>(scratch + align_up(sizeof(float) * R, 256) +
+                                                 align_up(sizeof(int32_t) * R, 256));
+  int* overflow = reinterpret_cast<int*>(reinterpret_cast<char*>(cta_tot) +
+                                         align_up(sizeof(int64_t) * (R / 8 + 1), 256));
+  uint32_t* mask = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(overflow) + 256);
+  uint8_t* vflag = reinterpret_cast<uint8_t*>(ws) + ws_bytes_for(p, sz, 1);
+  uint8_t* sflag = vflag + align_up(R, 256);
+  if (launch_plan(d, t, st, s) != cudaSuccess) return FPX_ERR_CUDA;
+  const int mw = static_cast<int>(mask_words(sz));
+  if (launch_vs_count(d, t, vert_bits, slash_bits, pattern_words(p), vflag, sflag, counts,
+                      cta_tot, mask, mw, s) != cudaSuccess)
+    return FPX_ERR_CUDA;
+  return launch_select_finish(d, row_ptr, col_idx, col_capacity, nnz_d, counts, cta_tot,
+                              overflow, mask, mw, t, st, s) == cudaSuccess
+             ? FPX_OK
+             : FPX_ERR_CUDA;
+}
+
+fpx_status fpx_vs_prefill(const fpx_problem* p, const void* q, const void* k, const void* v,
+                          const uint32_t* vert_bits, const uint32_t* slash_bits,
+                          const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
+                          void* ws, size_t ws_bytes, fpx_stream_t stream) {
+  Sizes sz;
+  fpx_status rc = check_problem(p, &sz);
+  if (rc != FPX_OK) return rc;
+  if (!attn_tc_supported(make_desc(p, sz), p->dtype)) return FPX_ERR_UNSUPPORTED;
+  if (p->total_tokens > 0 && (!vert_bits || !slash_bits)) return FPX_ERR_INVALID_ARG;
+  if (!aligned(vert_bits, 4) || !aligned(slash_bits, 4)) return FPX_ERR_ALIGNMENT;
+  return sparse_prefill_impl(p, q, k, v, nullptr, row_ptr, col_idx, o, lse, ws, ws_bytes, stream,
+                             vert_bits, slash_bits);
 }
 
 fpx_status fpx_sparse_prefill_paged(const fpx_problem* p, const void* q, const void* k_cache,

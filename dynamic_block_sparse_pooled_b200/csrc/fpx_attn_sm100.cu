@@ -7,6 +7,12 @@
 // The CTA walks the union of the two heads' CSR rows; a key block is loaded once (TMA, gathered
 // by block index) and multiplied only by the tile(s) that kept it.
 //
+// Persistent schedule: one CTA per SM; the load warp takes units from a queue that the order
+// kernel sorted by kept-tile count (heaviest first inside each KV head) and hands each to the
+// other roles through a two-slot ring in shared memory.  TMEM is allocated once per CTA; the
+// K / V rings, the S / P barriers and their phases run on across units, so the next unit's K / V
+// loads and S MMAs start while the previous unit's last softmax and epilogue finish.
+//
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for tile 0: one query row (= one TMEM lane) per thread
 //   warps 4-7  softmax for tile 1
@@ -58,23 +64,28 @@ constexpr int kLoadWarp = 10;
 constexpr uint32_t kSlotBytes = 32768;  // one 128 x 128 bf16 tile
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;    // lazy rescale threshold (log2 units)
-// shared memory: Q0, Q1, K slot 0/1, V slot 0/1 (32 KB each), then barriers
+// shared memory: Q0, Q1, K slot 0/1, V slot 0/1 (32 KB each), then barriers, the TMEM base
+// address, the abort flag and the two-slot unit ring
 constexpr uint32_t kOffQ = 0, kOffK = 2 * kSlotBytes, kOffV = 4 * kSlotBytes,
                    kOffBar = 6 * kSlotBytes;
 constexpr size_t kSmemBytes = 6 * kSlotBytes + 256 + 1024;
 
 enum Bar {
-  kBarQ = 0,
+  kBarQ = 0,        // Q tiles of the current unit landed (one phase per unit)
   kBarKFull = 1,    // +slot
   kBarKEmpty = 3,   // +slot
   kBarVFull = 5,    // +slot
   kBarVEmpty = 7,   // +slot
   kBarSFull = 9,    // +tile
   kBarPReady = 11,  // +tile
-  kBarODone = 13,   // +tile
+  kBarODone = 13,   // +tile: one phase per unit in which the tile had entries
   kBarDrain = 15,
-  kNumBars = 16
+  kBarQEmpty = 16,  // every S of the current unit completed (one phase per unit)
+  kBarUFull = 17,   // +slot: a unit index published in the ring
+  kBarUEmpty = 19,  // +slot: every reader took it
+  kNumBars = 21
 };
+constexpr int kUnitReaders = 9;  // the MMA warp and the eight softmax warps
 
 template <bool kFp8>
 struct Cfg {
@@ -212,14 +223,36 @@ __device__ __forceinline__ Unit decode_unit(const ProblemDesc& p, const int32_t*
   return w;
 }
 
-template <bool kFp8>
+// 128 bits [bit0, bit0 + 128) of a bitmask row of `words` words, as four words (bit c of the
+// result in word c / 32); bits outside the row read as 0.
+__device__ __forceinline__ void bits128(const uint32_t* __restrict__ row, int words, int64_t bit0,
+                                        uint32_t out[4]) {
+  const int64_t w0 = bit0 >> 5;  // floor, also for negative bit0
+  const int sh = static_cast<int>(bit0 & 31);
+  uint32_t wv[5];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) {
+    const int64_t wi = w0 + i;
+    wv[i] = (wi >= 0 && wi < words) ? __ldg(row + wi) : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) out[i] = __funnelshift_r(wv[i], wv[i + 1], sh);
+}
+
+// kMask: the vertical / slash token mask (query i of sequence s attends key j <= i iff bit
+// s_start + j of vbits[h] or bit s_start + (i - j) of sbits[h] is set) is applied inside every
+// listed key block, and a row that no key reaches gets O = 0, LSE = -inf.
+template <bool kFp8, bool kMask>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, ProblemDesc p,
                const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                __nv_bfloat16* __restrict__ o, float* __restrict__ lse, SeqTables tab,
-               const int32_t* __restrict__ order, StatusBlock* st) {
+               const int32_t* __restrict__ order, int* __restrict__ queue_head, int n_units,
+               const uint32_t* __restrict__ vbits, const uint32_t* __restrict__ sbits, int words,
+               StatusBlock* st) {
   using C = Cfg<kFp8>;
+  constexpr unsigned kFull = 0xffffffffu;
   if (!*tab.valid) return;  // inconsistent cu_seqlens (recorded by the plan kernel)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -228,13 +261,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t bar0 = sbase + kOffBar;  // barrier i at bar0 + 8 * i
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 8 * kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * kNumBars + 4);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * kNumBars + 8);
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const Unit w = decode_unit(p, tab.blk_base, row_ptr, order ? order[blockIdx.x] : blockIdx.x);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     mbar_init(bar(kBarQ), 1);
+    mbar_init(bar(kBarQEmpty), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarKFull + i), 1);
       mbar_init(bar(kBarKEmpty + i), 1);
@@ -243,6 +277,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarPReady + i), kTileM / 32);  // one arrival per softmax warp
       mbar_init(bar(kBarODone + i), 1);
+      mbar_init(bar(kBarUFull + i), 1);
+      mbar_init(bar(kBarUEmpty + i), kUnitReaders);
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -256,24 +292,61 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // Unit k of this CTA sits in ring slot k & 1; its readers (the MMA warp and the eight softmax
+  // warps, each fully converged here) release the slot once they have read it.  -1 ends the
+  // loop.  The wait is warp-uniform, so a timeout takes the whole warp out together.
+  auto take_unit = [&](int k, int& u) -> bool {
+    const uint32_t b = bar(kBarUFull + (k & 1));
+    if (!__all_sync(kFull, mbar_wait(b, (k >> 1) & 1, abort_flag))) return false;
+    u = unit_ring[k & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(kBarUEmpty + (k & 1)));
+    return true;
+  };
+
   if (warp >= 8) {
   setmaxnreg_dec<kOtherRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer ----
-    // Warp-uniform loop; one elected lane issues the copies.
-    constexpr unsigned kFull = 0xffffffffu;
+    // Takes units from the queue (heaviest first), publishes each to the other roles, then
+    // loads its Q tiles and the K / V blocks of the union of its two CSR rows into the rings.
+    // Warp-uniform loop; lane 0 / one elected lane issue.
     if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    RowMerge m(col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I);
-    RowMerge peek = m;
-    int J, uses;
-    int n = 0;
-    bool q_issued = false;
-    if (peek.next(J, uses)) {
-      q_issued = true;
+    int n = 0;        // K / V ring entries issued (over all units)
+    int k = 0;        // units published
+    int q_loads = 0;  // units whose Q tiles were requested
+    bool ok = true;
+    while (true) {
+      int u = -1;
+      if (lane == 0) {
+        const int qi = atomicAdd(queue_head, 1);
+        u = qi < n_units ? order[qi] : -1;
+      }
+      u = __shfl_sync(kFull, u, 0);
+      if (!__all_sync(kFull, mbar_wait(bar(kBarUEmpty + (k & 1)), ((k >> 1) & 1) ^ 1,
+                                       abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        unit_ring[k & 1] = u;
+        mbar_arrive(bar(kBarUFull + (k & 1)));  // release: the slot write is visible first
+      }
+      __syncwarp();
+      ++k;
+      if (u < 0) break;
+      const Unit w = decode_unit(p, tab.blk_base, row_ptr, u);
+      // Q tiles of this unit (every unit has them, with or without entries): the buffers are
+      // free once every S of the previous unit has completed
+      if (k > 1 && !__all_sync(kFull, mbar_wait(bar(kBarQEmpty), (k - 2) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
       if (elect_one()) {
         mbar_arrive_expect_tx(bar(kBarQ), C::kTileBytes * w.ntiles);
 #pragma unroll
@@ -285,59 +358,67 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         bx * 128 / C::kElem, w.h[t], w.tok0 + w.I * kTileM);
         }
       }
-    }
-    while (m.next(J, uses)) {
-      const int slot = n & 1;
-      const uint32_t ph = (n >> 1) & 1;
-      // first K / V row of block J (its page when K / V are paged); a page index outside the
-      // cache is recorded and read past the end of the map (TMA fills zeros there)
-      int64_t kv_row = kv_block_row(p, w.s, J, w.tok0);
-      if (kv_row < 0) {
-        if (elect_one()) record_error(st, FPX_ERR_DEVICE_INPUT, 34, w.s, J);
-        kv_row = static_cast<int64_t>(p.num_pages) * kTileN;
-      }
-      const int kv_tok = static_cast<int>(kv_row);
-      if (!__all_sync(kFull, mbar_wait(bar(kBarKEmpty + slot), ph ^ 1, abort_flag))) break;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(kBarKFull + slot), C::kTileBytes);
+      ++q_loads;
+      RowMerge m(col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I);
+      int J, uses;
+      while (m.next(J, uses)) {
+        const int slot = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        // first K / V row of block J (its page when K / V are paged); a page index outside the
+        // cache is recorded and read past the end of the map (TMA fills zeros there)
+        int64_t kv_row = kv_block_row(p, w.s, J, w.tok0);
+        if (kv_row < 0) {
+          if (elect_one()) record_error(st, FPX_ERR_DEVICE_INPUT, 34, w.s, J);
+          kv_row = static_cast<int64_t>(p.num_pages) * kTileN;
+        }
+        const int kv_tok = static_cast<int>(kv_row);
+        if (!__all_sync(kFull, mbar_wait(bar(kBarKEmpty + slot), ph ^ 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(kBarKFull + slot), C::kTileBytes);
 #pragma unroll
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(sbase + kOffK + slot * kSlotBytes + bx * C::kBoxBytes, &tmK,
-                      bar(kBarKFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
-      }
-      if (!__all_sync(kFull, mbar_wait(bar(kBarVEmpty + slot), ph ^ 1, abort_flag))) {
-        // K of this entry is in flight; only its K barrier is drained below
-        volatile int never = 0;
-        mbar_wait(bar(kBarKFull + slot), ph, &never);
-        break;
-      }
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(kBarVFull + slot), C::kTileBytes);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(sbase + kOffK + slot * kSlotBytes + bx * C::kBoxBytes, &tmK,
+                        bar(kBarKFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
+        }
+        if (!__all_sync(kFull, mbar_wait(bar(kBarVEmpty + slot), ph ^ 1, abort_flag))) {
+          // K of this entry is in flight; only its K barrier is drained below
+          volatile int never = 0;
+          mbar_wait(bar(kBarKFull + slot), ph, &never);
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(kBarVFull + slot), C::kTileBytes);
 #pragma unroll
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(sbase + kOffV + slot * kSlotBytes + bx * C::kBoxBytes, &tmV,
-                      bar(kBarVFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(sbase + kOffV + slot * kSlotBytes + bx * C::kBoxBytes, &tmV,
+                        bar(kBarVFull + slot), bx * 128 / C::kElem, w.kvh, kv_tok);
+        }
+        ++n;
       }
-      ++n;
+      if (!ok) break;
     }
-    // Drain: wait (bounded) until every load this warp issued has landed.  On the normal path
-    // each of these has already completed.
+    if (!ok) *abort_flag = 1;
+    // Drain: wait (bounded) until every load this warp issued has landed: the last Q (one Q
+    // load at most is in flight) and the last two ring entries.
     volatile int never = 0;
-    if (q_issued) mbar_wait(bar(kBarQ), 0, &never);
-    for (int k = n - 2; k < n; ++k) {
-      if (k < 0) continue;
-      const int slot = k & 1;
-      const uint32_t ph = (k >> 1) & 1;
+    if (q_loads > 0) mbar_wait(bar(kBarQ), (q_loads - 1) & 1, &never);
+    for (int e = n - 2; e < n; ++e) {
+      if (e < 0) continue;
+      const int slot = e & 1;
+      const uint32_t ph = (e >> 1) & 1;
       mbar_wait(bar(kBarKFull + slot), ph, &never);
       mbar_wait(bar(kBarVFull + slot), ph, &never);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer -------
     // Warp-uniform sequential loop; one elected lane issues and commits.  Order per union entry
-    // n:  S_0(n) | O_1 += P_1(n') V_n' (tile 1's previous entry) | S_1(n) | O_0 += P_0(n) V_n.
+    // n:  O_1 += P_1(n') V_n' (tile 1's previous entry), S_1(n) | O_0 += P_0(n) V_n, S_0(n + 1).
     // Softmax 0 of entry n runs while the tensor pipe executes tile 1's P*V and S, and softmax 1
     // while it executes tile 0's P*V and next S, so the two softmaxes alternate.
-    constexpr unsigned kFull = 0xffffffffu;
     // Matrix descriptors of every buffer, built once.  A k-step inside a buffer only moves the
     // start-address field (bits 0-13, address >> 4): a constant add to the descriptor.
     const uint64_t qdesc0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
@@ -365,113 +446,130 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         else mma_f16_ts(tO, tS + kk * 8, bd, C::kIdescPV, acc);
       }
     };
-    RowMerge m(col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I);
-    int J, uses;
-    bool have = m.next(J, uses);
-    bool ok = true;
-    if (have) ok = __all_sync(kFull, mbar_wait(bar(kBarQ), 0, abort_flag));
+    int n = 0;  // ring entries consumed (over all units)
+    int k = 0;  // units taken
     uint32_t p_phase0 = 0, p_phase1 = 0;
-    bool o0_started = false, o1_started = false;
-    int pend = -1;  // union index of tile 1's entry whose P*V is not issued yet
-    int n = 0;
-    // A P*V and the S that follows it in the same tile are issued back to back from one elected
-    // block: any wait or bookkeeping between them would leave the tensor pipe idle.
-    if (ok && have) {  // S_0 of the first entry
-      if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + 0), 0, abort_flag))) {
-        ok = false;
-      } else {
+    bool ok = true;
+    while (ok) {
+      int u;
+      if (!take_unit(k, u)) { ok = false; break; }
+      ++k;
+      if (u < 0) break;
+      const Unit w = decode_unit(p, tab.blk_base, row_ptr, u);
+      RowMerge m(col_idx, w.beg[0], w.end[0], w.beg[1], w.end[1], w.I);
+      int J, uses;
+      bool have = m.next(J, uses);
+      if (!__all_sync(kFull, mbar_wait(bar(kBarQ), (k - 1) & 1, abort_flag))) { ok = false; break; }
+      bool o0_started = false, o1_started = false;
+      int pend = -1;  // ring index of tile 1's entry whose P*V is not issued yet
+      // A P*V and the S that follows it in the same tile are issued back to back from one
+      // elected block: any wait or bookkeeping between them would leave the tensor pipe idle.
+      if (have) {  // S_0 of the first entry
+        if (!__all_sync(kFull, mbar_wait(bar(kBarKFull + (n & 1)), (n >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
         if (elect_one() && (uses & 1)) {
           tc_fence_after();
-          issue_s(tS0, qdesc0, 0);
+          issue_s(tS0, qdesc0, n & 1);
           mma_commit(bar(kBarSFull + 0));
         }
         __syncwarp();
       }
-    }
-    while (ok && have) {
-      const int slot = n & 1;
-      const uint32_t ph = (n >> 1) & 1;
-      // tile 1: O_1 += P_1 V of its previous entry, then S_1 of this entry
-      const bool pv1 = pend >= 0;
-      const int ps = pend & 1;
-      if (pv1) {
-        if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag))) { ok = false; break; }
-        p_phase1 ^= 1;
-        if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), (pend >> 1) & 1, abort_flag))) { ok = false; break; }
-      }
-      if (elect_one()) {
-        tc_fence_after();
+      while (have) {
+        const int slot = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        // tile 1: O_1 += P_1 V of its previous entry, then S_1 of this entry
+        const bool pv1 = pend >= 0;
+        const int ps = pend & 1;
         if (pv1) {
-          issue_pv(tO1, tS1, ps, o1_started);
-          mma_commit(bar(kBarVEmpty + ps));
+          if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag))) { ok = false; break; }
+          p_phase1 ^= 1;
+          if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), (pend >> 1) & 1, abort_flag))) { ok = false; break; }
         }
-        if (uses & 2) {
-          issue_s(tS1, qdesc1, slot);
-          mma_commit(bar(kBarSFull + 1));
+        if (elect_one()) {
+          tc_fence_after();
+          if (pv1) {
+            issue_pv(tO1, tS1, ps, o1_started);
+            mma_commit(bar(kBarVEmpty + ps));
+          }
+          if (uses & 2) {
+            issue_s(tS1, qdesc1, slot);
+            mma_commit(bar(kBarSFull + 1));
+          }
+          mma_commit(bar(kBarKEmpty + slot));  // every S reading K_n has been issued
         }
-        mma_commit(bar(kBarKEmpty + slot));  // every S reading K_n has been issued
-      }
-      __syncwarp();
-      if (pv1) {
-        o1_started = true;
-        pend = -1;
-      }
-      // The next union entry (global loads of the CSR arrays) and its K tile, while this entry's
-      // MMAs run and softmax 0 works.
-      int uses_next = 0;
-      const bool have_next = m.next(J, uses_next);
-      const int nslot = (n + 1) & 1;
-      if (have_next &&
-          !__all_sync(kFull, mbar_wait(bar(kBarKFull + nslot), ((n + 1) >> 1) & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      const bool s0_next = have_next && (uses_next & 1);
-      // tile 0: O_0 += P_0 V of this entry, then S_0 of the next entry
-      if (uses & 1) {
-        if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 0), p_phase0, abort_flag))) { ok = false; break; }
-        p_phase0 ^= 1;
-        if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + slot), ph, abort_flag))) { ok = false; break; }
-      }
-      if (elect_one()) {
-        tc_fence_after();
+        __syncwarp();
+        if (pv1) {
+          o1_started = true;
+          pend = -1;
+        }
+        // The next union entry (global loads of the CSR arrays) and its K tile, while this
+        // entry's MMAs run and softmax 0 works.
+        int uses_next = 0;
+        const bool have_next = m.next(J, uses_next);
+        const int nslot = (n + 1) & 1;
+        if (have_next &&
+            !__all_sync(kFull, mbar_wait(bar(kBarKFull + nslot), ((n + 1) >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const bool s0_next = have_next && (uses_next & 1);
+        // tile 0: O_0 += P_0 V of this entry, then S_0 of the next entry
         if (uses & 1) {
-          issue_pv(tO0, tS0, slot, o0_started);
-          if (!(uses & 2)) mma_commit(bar(kBarVEmpty + slot));
+          if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 0), p_phase0, abort_flag))) { ok = false; break; }
+          p_phase0 ^= 1;
+          if (!__all_sync(kFull, mbar_wait(bar(kBarVFull + slot), ph, abort_flag))) { ok = false; break; }
         }
-        if (s0_next) {
-          issue_s(tS0, qdesc0, nslot);
-          mma_commit(bar(kBarSFull + 0));
+        if (elect_one()) {
+          tc_fence_after();
+          if (uses & 1) {
+            issue_pv(tO0, tS0, slot, o0_started);
+            if (!(uses & 2)) mma_commit(bar(kBarVEmpty + slot));
+          }
+          if (s0_next) {
+            issue_s(tS0, qdesc0, nslot);
+            mma_commit(bar(kBarSFull + 0));
+          }
         }
+        __syncwarp();
+        if (uses & 1) o0_started = true;
+        if (uses & 2) pend = n;
+        ++n;
+        have = have_next;
+        uses = uses_next;
       }
+      if (!ok) break;
+      // every S of this unit is issued: Q may be reloaded once they complete
+      if (elect_one()) mma_commit(bar(kBarQEmpty));
       __syncwarp();
-      if (uses & 1) o0_started = true;
-      if (uses & 2) pend = n;
-      ++n;
-      have = have_next;
-      uses = uses_next;
-    }
-    if (ok && pend >= 0) {  // tile 1's last P*V
-      const int ps = pend & 1;
-      if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag)) ||
-          !__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), (pend >> 1) & 1, abort_flag))) {
-        ok = false;
-      } else {
+      if (pend >= 0) {  // tile 1's last P*V
+        const int ps = pend & 1;
+        if (!__all_sync(kFull, mbar_wait(bar(kBarPReady + 1), p_phase1, abort_flag)) ||
+            !__all_sync(kFull, mbar_wait(bar(kBarVFull + ps), (pend >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        p_phase1 ^= 1;
         if (elect_one()) {
           tc_fence_after();
           issue_pv(tO1, tS1, ps, o1_started);
           mma_commit(bar(kBarVEmpty + ps));
         }
         __syncwarp();
+        o1_started = true;
       }
+      // O_t is final once its P*V complete; a tile without entries gets no commit (its softmax
+      // warps do not wait for one)
+      if (elect_one()) {
+        if (o0_started) mma_commit(bar(kBarODone + 0));
+        if (o1_started) mma_commit(bar(kBarODone + 1));
+      }
+      __syncwarp();
     }
     if (!ok) *abort_flag = 1;
-    if (elect_one()) {
-      mma_commit(bar(kBarODone + 0));
-      mma_commit(bar(kBarODone + 1));
-      // drain: every MMA issued by this warp completes before TMEM can be released
-      mma_commit(bar(kBarDrain));
-    }
+    // drain: every MMA issued by this warp completes before TMEM can be released
+    if (elect_one()) mma_commit(bar(kBarDrain));
     volatile int never = 0;
     mbar_wait(bar(kBarDrain), 0, &never);
   }
@@ -480,32 +578,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ------------------------------------------------------------------ softmax ----------
     const int t = warp >> 2;                 // tile
     const int row = tid & 127;               // query row = TMEM lane
-    const int my_h = t ? w.h[1] : w.h[0];
-    const int my_r = t ? w.r[1] : w.r[0];
-    const int my_beg = t ? w.beg[1] : w.beg[0];
-    const int my_end = t ? w.end[1] : w.end[0];
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + t * 128 + lane_base;
     const uint32_t tO = tmem + 256 + t * 128 + lane_base;
-    const int qpos = w.I * kTileM + row;
-    const bool write = t < w.ntiles && qpos < w.n_s;
-    const int64_t tq = static_cast<int64_t>(w.tok0) + qpos;
-    float sl2 = p.scale * 1.4426950408889634f;
-    float vsc = 1.f;
-    if (kFp8 && t < w.ntiles) {
-      sl2 *= p.q_scale[my_h] * p.k_scale[w.kvh];
-      vsc = p.v_scale[w.kvh];
-    }
-    float m_ref = -CUDART_INF_F, l_run = 0.f;
-    uint32_t s_phase = 0;
-    int it = 0;
+    uint32_t s_phase = 0;   // S_t phases (over all units)
+    uint32_t od_phase = 0;  // O_t-done phases: one per unit in which this tile had entries
+    int k = 0;
+    int my_r = -1, it = 0;
     bool ok = true;
-    if (t < w.ntiles) {
-      for (int e = my_beg; e < my_end; ++e) {
+    while (ok) {
+      int u;
+      if (!take_unit(k, u)) { ok = false; break; }
+      ++k;
+      if (u < 0) break;
+      const Unit w = decode_unit(p, tab.blk_base, row_ptr, u);
+      if (t >= w.ntiles) continue;
+      const int my_h = w.h[t];
+      my_r = w.r[t];
+      const int qpos = w.I * kTileM + row;
+      const bool write = qpos < w.n_s;
+      const int64_t tq = static_cast<int64_t>(w.tok0) + qpos;
+      float sl2 = p.scale * 1.4426950408889634f;
+      float vsc = 1.f;
+      if (kFp8) {
+        sl2 *= p.q_scale[my_h] * p.k_scale[w.kvh];
+        vsc = p.v_scale[w.kvh];
+      }
+      float m_ref = -CUDART_INF_F, l_run = 0.f;
+      const uint32_t* vrow = kMask ? vbits + static_cast<int64_t>(my_h) * words : nullptr;
+      const uint32_t* srow = kMask ? sbits + static_cast<int64_t>(my_h) * words : nullptr;
+      it = 0;
+      for (int e = w.beg[t]; e < w.end[t]; ++e) {
         const int J = col_idx[e];
         if (J < 0 || J > w.I) {
           if (row == 0) record_error(st, FPX_ERR_DEVICE_INPUT, 30, my_r, J);
           continue;
+        }
+        // token mask of this row in block J: verticals (bit c = key J*B + c) or slashes (bit
+        // c = offset qpos - J*B - c, the 128 offsets read reversed)
+        uint32_t am[4];
+        if (kMask) {
+          uint32_t vm[4], xs[4];
+          bits128(vrow, words, static_cast<int64_t>(w.tok0) + J * kTileN, vm);
+          bits128(srow, words, static_cast<int64_t>(w.tok0) + qpos - J * kTileN - (kTileN - 1), xs);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) am[i] = vm[i] | __brev(xs[3 - i]);
         }
         if (!mbar_wait(bar(kBarSFull + t), s_phase, abort_flag)) { ok = false; break; }
         s_phase ^= 1;
@@ -525,6 +642,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int j = 0; j < 64; ++j)
             if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
         }
+        if (kMask) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            if (!((am[j >> 5] >> (j & 31)) & 1u)) r[j] = __float_as_uint(-CUDART_INF_F);
+        }
         const float mx_lo = row_max64(r);
         tmem_wait_ld(r + 64);
         tmem_wait_ld(r + 96);
@@ -533,7 +655,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int j = 64; j < 128; ++j)
             if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
         }
-        const float mx = fmaxf(mx_lo, row_max64(r + 64)) * sl2;  // finite: key 0 is always visible
+        if (kMask) {
+#pragma unroll
+          for (int j = 64; j < 128; ++j)
+            if (!((am[j >> 5] >> (j & 31)) & 1u)) r[j] = __float_as_uint(-CUDART_INF_F);
+        }
+        // finite unless kMask: key 0 of a block row is always visible without the token mask;
+        // with it a row may see no key yet (m_ref = -inf), and -inf then stands for "none"
+        const float mx = fmaxf(mx_lo, row_max64(r + 64)) * sl2;
         // lazy rescale: move the reference max only when the block max exceeds it by > 2^8
         float corr = 1.f;
         if (mx > m_ref + kRescaleLog2) {
@@ -555,10 +684,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         // P = exp2(s * sl2 - m_ref), packed in place and written over S
         // first half of P stored while the second half is computed
-        float rs = softmax_part_to_p<kFp8, 0, 64>(r, sl2, -m_ref);
+        // (a row that no key has reached yet: exponents of -inf, P = 0, and the weights the
+        // FMA-pipe exp2 gives them are cleared by the rescale that its first key triggers)
+        const float neg_m = (kMask && m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+        float rs = softmax_part_to_p<kFp8, 0, 64>(r, sl2, neg_m);
         if (kFp8) tmem_st16(tS, r);
         else tmem_st32(tS, r);
-        rs += softmax_part_to_p<kFp8, 64, 64>(r, sl2, -m_ref);
+        rs += softmax_part_to_p<kFp8, 64, 64>(r, sl2, neg_m);
         if (kFp8) tmem_st16(tS + 16, r + 16);
         else tmem_st32(tS + 32, r + 32);
         l_run += rs;
@@ -568,42 +700,50 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if ((tid & 31) == 0) mbar_arrive(bar(kBarPReady + t));
         ++it;
       }
+      if (!ok) break;
       // epilogue: wait for the last P*V, normalise, store O (bf16) and the natural-log LSE
-      if (ok && it > 0 && !mbar_wait(bar(kBarODone + t), 0, abort_flag)) ok = false;
-      if (!ok) {
-        *abort_flag = 1;
-        if (row == 0) record_error(st, FPX_ERR_TIMEOUT, 31, my_r, it);
-      } else {
-        tc_fence_after();
-        uint4* orow = reinterpret_cast<uint4*>(o + (tq * p.hq + my_h) * kHeadDim);
-        if (it == 0) {
-          if (write) {
+      uint4* orow = reinterpret_cast<uint4*>(o + (tq * p.hq + my_h) * kHeadDim);
+      if (it == 0) {
+        if (write) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
-            if (lse) lse[static_cast<int64_t>(my_h) * p.total_tokens + tq] = -CUDART_INF_F;
-          }
-        } else {
-          const float inv = vsc / l_run;
+          for (int i = 0; i < 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
+          if (lse) lse[static_cast<int64_t>(my_h) * p.total_tokens + tq] = -CUDART_INF_F;
+        }
+        continue;
+      }
+      if (!mbar_wait(bar(kBarODone + t), od_phase, abort_flag)) { ok = false; break; }
+      od_phase ^= 1;
+      tc_fence_after();
+      // kMask: a row that no key reached (blocks were listed, the token mask removed every key
+      // of them for this row) gets O = 0 and LSE = -inf; every lane still takes part in the
+      // warp-wide TMEM loads below
+      const bool none = kMask && m_ref == -CUDART_INF_F;
+      const float inv = none ? 0.f : vsc / l_run;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + c * 32, r);
-            tmem_wait_ld(r);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + c * 32, r);
+        tmem_wait_ld(r);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 v4;
-              v4.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
-              v4.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
-              v4.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
-              v4.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
-              if (write) orow[c * 4 + i] = v4;
-            }
-          }
-          if (lse && write)
-            lse[static_cast<int64_t>(my_h) * p.total_tokens + tq] =
-                (m_ref + __log2f(l_run)) * 0.6931471805599453f;
+        for (int i = 0; i < 4; ++i) {
+          uint4 v4;
+          v4.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+          v4.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+          v4.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+          v4.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+          if (write) orow[c * 4 + i] = v4;
         }
       }
+      if (lse && write)
+        lse[static_cast<int64_t>(my_h) * p.total_tokens + tq] =
+            none ? -CUDART_INF_F : (m_ref + __log2f(l_run)) * 0.6931471805599453f;
+      // O_t's TMEM columns are read: the next unit's first P*V into them waits for this warp's
+      // first P of that unit, which comes after these loads in program order
+      tc_fence_before();
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (row == 0) record_error(st, FPX_ERR_TIMEOUT, 31, my_r, it);
     }
   }
 
@@ -666,10 +806,26 @@ int64_t attn_tc_units(const ProblemDesc& p) {
   return static_cast<int64_t>(p.hkv) * p.nb_total * ((p.group + 1) / 2);
 }
 
+// Streaming multiprocessors of the current device (one resident CTA each: the kernel's shared
+// memory admits no second one), looked up once per device.
+static int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      return 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
 cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                            const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                            void* o, float* lse, SeqTables t, const int32_t* order,
-                           StatusBlock* st, cudaStream_t s, bool* encode_failed) {
+                           int* queue_head, const uint32_t* vbits, const uint32_t* sbits,
+                           int words, StatusBlock* st, cudaStream_t s, bool* encode_failed) {
   using namespace sm100;
   *encode_failed = false;
   const int64_t units = attn_tc_units(p);
@@ -683,12 +839,17 @@ cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, co
     *encode_failed = true;
     return cudaErrorInvalidValue;
   }
-  auto kern = fp8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  const bool mask = vbits != nullptr;
+  auto kern = fp8 ? (mask ? attn_tc_kernel<true, true> : attn_tc_kernel<true, false>)
+                  : (mask ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(units), kThreads, kSmemBytes, s>>>(
-      mq, mk, mv, p, row_ptr, col_idx, static_cast<__nv_bfloat16*>(o), lse, t, order, st);
+  // persistent: one CTA per SM takes units from the queue (heaviest first) until it is empty
+  const int64_t grid = units < sm_count() ? units : sm_count();
+  kern<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(
+      mq, mk, mv, p, row_ptr, col_idx, static_cast<__nv_bfloat16*>(o), lse, t, order, queue_head,
+      static_cast<int>(units), vbits, sbits, words, st);
   return cudaGetLastError();
 }
 

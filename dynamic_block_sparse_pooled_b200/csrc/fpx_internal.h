@@ -47,18 +47,45 @@ int select_ctas(const ProblemDesc& p);
 bool make_tmap_rows128(CUtensorMap* map, const void* base, int T, int H, int D, int elem_bytes);
 
 // fpx_sparse_prefill: tile schedule, then one of the two attention kernels.
-// `units`: schedule the tensor-core kernel's two-head units instead of single CSR rows.
-cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, bool units,
-                         cudaStream_t s);
+// `units`: schedule the tensor-core kernel's two-head units instead of single CSR rows.  The
+// items are sorted by their kept-tile counts in row_ptr (heaviest first inside each KV head);
+// *queue_head is reset to 0 for the persistent kernel's work queue.  nb_max = blocks of the
+// longest sequence.
+cudaError_t launch_order(const ProblemDesc& p, int nb_max, SeqTables t, const int32_t* row_ptr,
+                         int32_t* order, int* queue_head, bool units, cudaStream_t s);
 cudaError_t launch_attn_simt(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              void* o, float* lse, SeqTables t, const int32_t* order,
                              StatusBlock* st, cudaStream_t s);
 bool attn_tc_supported(const ProblemDesc& p, fpx_dtype dt);
 // Returns cudaSuccess or the first error; `encode_failed` is set if a tensor map was rejected.
+// vbits / sbits non-null: the vertical / slash token mask (uint32 [hq][words]) is applied.
 cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
                            const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                            void* o, float* lse, SeqTables t, const int32_t* order,
-                           StatusBlock* st, cudaStream_t s, bool* encode_failed);
+                           int* queue_head, const uint32_t* vbits, const uint32_t* sbits,
+                           int words, StatusBlock* st, cudaStream_t s, bool* encode_failed);
+
+// Query-probe vertical / slash discovery (fpx_probe.cu): zeroes and fills the two bitmasks
+// (uint32 [hq][words]).  chunk_base: [num_seqs + 1] int32; partial: float2 [total_chunks * hkv *
+// probe_tiles * 128]; bound: float2 [num_seqs * hq * n_probe].
+int probe_tiles(const ProblemDesc& p, int n_probe);
+size_t probe_smem(int tiles);
+cudaError_t launch_probe(const ProblemDesc& p, fpx_dtype dt, const void* q, const void* k,
+                         int n_probe, float alpha_v, float alpha_s, int chunk_blocks,
+                         int total_chunks, SeqTables t, int32_t* chunk_base, float2* partial,
+                         float2* bound, uint32_t* vbits, uint32_t* sbits, int words,
+                         StatusBlock* st, cudaStream_t s, bool* encode_failed);
+// Candidate key blocks of the vertical / slash attention into the select stage's keep bitmask
+// and counts (then launch_select_finish builds the CSR).  vflag / sflag: uint8 [hq * NB] each.
+cudaError_t launch_vs_count(const ProblemDesc& p, SeqTables t, const uint32_t* vbits,
+                            const uint32_t* sbits, int words, uint8_t* vflag, uint8_t* sflag,
+                            int32_t* counts, int64_t* cta_tot, uint32_t* mask, int mask_words,
+                            cudaStream_t s);
+// The scan and emit kernels of the select stage on counts / mask written by a count kernel.
+cudaError_t launch_select_finish(const ProblemDesc& p, int32_t* row_ptr, int32_t* col_idx,
+                                 int64_t capacity, int64_t* nnz_d, const int32_t* counts,
+                                 int64_t* cta_tot, int* overflow, const uint32_t* mask,
+                                 int mask_words, SeqTables t, StatusBlock* st, cudaStream_t s);
 
 }  // namespace fpx

@@ -732,6 +732,21 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
 
 int select_ctas(const ProblemDesc& p) { return (p.hq * p.nb_total + kSelRows - 1) / kSelRows; }
 
+cudaError_t launch_select_finish(const ProblemDesc& p, int32_t* row_ptr, int32_t* col_idx,
+                                 int64_t capacity, int64_t* nnz_d, const int32_t* counts,
+                                 int64_t* cta_tot, int* overflow, const uint32_t* mask,
+                                 int mask_words, SeqTables t, StatusBlock* st, cudaStream_t s) {
+  const int R = p.hq * p.nb_total;
+  const int nblk = select_ctas(p);
+  select_scan_kernel<<<1, kScanThreads, 0, s>>>(R, nblk, cta_tot, row_ptr, capacity, nnz_d,
+                                                overflow, t.valid, st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || R == 0) return e;
+  select_emit_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, counts, cta_tot, row_ptr, col_idx,
+                                                     overflow, mask, mask_words, t);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha, int sink,
                           int window, int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
                           int64_t* nnz_d, float* rowmax, int32_t* counts, int64_t* cta_tot,
@@ -757,53 +772,120 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
 }
 
 // ------------------------------------------------------------------------------------------
-// order: the attention schedule.  Items are grouped by KV head (so the CTAs resident at any
-// moment share K/V blocks through L2) and, inside a group, heaviest first (largest local block
-// index I first, since a row can keep at most I + 1 blocks), then sequence, then slot:
-//   pos = kvh*slots*NB + slots*sum_s' max(0, nb_s' - 1 - I) + slots*#{s' < s : nb_s' > I} + sub
-// Rows (CUDA-core kernel): item r = h*NB + b, slots = Hq/Hkv, sub = h % slots.
-// Units (tensor-core kernel, two Q heads of one KV group): item u = (kvh*NB + b)*slots + sub
-// with slots = ceil((Hq/Hkv) / 2), sub = the head pair.
+// order: the attention schedule, from the CSR the attention will read.  Items are grouped by KV
+// head (so the CTAs resident at any moment share K/V blocks through L2) and, inside a group,
+// sorted by their real cost, heaviest first (longest-processing-time order, so that the last
+// items to start are the short ones): cost = the kept tiles of the item's CSR rows.
+// Rows (CUDA-core kernel): item r = h*NB + b.  Units (tensor-core kernel, two Q heads of one KV
+// group at one query block): item u = (kvh*NB + b)*slots + pair, slots = ceil((Hq/Hkv) / 2).
+// One CTA runs a counting sort over (KV head, cost bucket) bins in shared memory; the order of
+// items inside one bin is arbitrary (it changes where, not what, each item computes).  It also
+// resets the work-queue head that the persistent attention kernel takes items from.
 // ------------------------------------------------------------------------------------------
-__global__ void order_kernel(ProblemDesc p, const int32_t* __restrict__ blk_base,
-                             const int32_t* __restrict__ valid, int32_t* __restrict__ order,
-                             int units) {
-  if (!*valid) return;
-  const int slots = units ? (p.group + 1) / 2 : p.group;
-  const int n_items = p.hkv * p.nb_total * slots;
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n_items) return;
-  int kvh, b, sub;
-  if (units) {
-    kvh = i / (p.nb_total * slots);
-    const int rem = i - kvh * p.nb_total * slots;
-    b = rem / slots;
-    sub = rem - b * slots;
-  } else {
-    const int h = i / p.nb_total;
-    b = i - h * p.nb_total;
-    kvh = h / p.group;
-    sub = h - kvh * p.group;
-  }
-  const int s = seq_of_block(blk_base, p.num_seqs, b);
-  const int I = b - blk_base[s];
-  int64_t heavier = 0, same_earlier = 0;
-  for (int s2 = 0; s2 < p.num_seqs; ++s2) {
-    const int nb2 = blk_base[s2 + 1] - blk_base[s2];
-    heavier += max(0, nb2 - 1 - I);
-    if (s2 < s && nb2 > I) ++same_earlier;
-  }
-  const int64_t pos = static_cast<int64_t>(kvh) * slots * p.nb_total + slots * heavier +
-                      slots * same_earlier + sub;
-  order[pos] = i;
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderMaxBins = 16384;  // 64 KB of shared-memory histogram
+
+struct OrderShape {
+  int slots, per_kv, n_items, nbk, cost_cap, kvb;  // kvb: KV-head groups (<= kOrderMaxBins)
+};
+
+inline OrderShape order_shape(const ProblemDesc& p, int nb_max, bool units) {
+  OrderShape o;
+  o.slots = units ? (p.group + 1) / 2 : p.group;
+  o.per_kv = p.nb_total * o.slots;
+  o.n_items = p.hkv * o.per_kv;
+  o.cost_cap = (units ? 2 : 1) * nb_max;
+  o.kvb = p.hkv < kOrderMaxBins ? p.hkv : kOrderMaxBins;
+  const int cap_bins = kOrderMaxBins / o.kvb;
+  o.nbk = o.cost_cap + 1 < cap_bins ? o.cost_cap + 1 : cap_bins;
+  return o;
 }
 
-cudaError_t launch_order(const ProblemDesc& p, SeqTables t, int32_t* order, bool units,
-                         cudaStream_t s) {
-  const int slots = units ? (p.group + 1) / 2 : p.group;
-  const int n_items = p.hkv * p.nb_total * slots;
-  if (n_items == 0) return cudaSuccess;
-  order_kernel<<<(n_items + 255) / 256, 256, 0, s>>>(p, t.blk_base, t.valid, order, units ? 1 : 0);
+// (KV head, cost) of item i; the bin sorts heavier items first inside a KV head.
+__device__ __forceinline__ int order_bin(const ProblemDesc& p, const OrderShape& o,
+                                         const int32_t* __restrict__ row_ptr, int i, int units) {
+  int kvh, cost;
+  if (units) {
+    kvh = i / o.per_kv;
+    const int rem = i - kvh * o.per_kv;
+    const int b = rem / o.slots;
+    const int pair = rem - b * o.slots;
+    const int h0 = kvh * p.group + 2 * pair;
+    const int r0 = h0 * p.nb_total + b;
+    cost = __ldg(row_ptr + r0 + 1) - __ldg(row_ptr + r0);
+    if (2 * pair + 1 < p.group) {
+      const int r1 = r0 + p.nb_total;
+      cost += __ldg(row_ptr + r1 + 1) - __ldg(row_ptr + r1);
+    }
+  } else {
+    const int h = i / p.nb_total;
+    kvh = h / p.group;
+    cost = __ldg(row_ptr + i + 1) - __ldg(row_ptr + i);
+  }
+  cost = min(max(cost, 0), o.cost_cap);
+  const int bucket = static_cast<int>(static_cast<int64_t>(cost) * o.nbk / (o.cost_cap + 1));
+  const int kvg = static_cast<int>(static_cast<int64_t>(kvh) * o.kvb / p.hkv);
+  return kvg * o.nbk + (o.nbk - 1 - bucket);
+}
+
+__global__ void __launch_bounds__(kOrderThreads) order_kernel(
+    ProblemDesc p, const int32_t* __restrict__ valid, const int32_t* __restrict__ row_ptr,
+    int32_t* __restrict__ order, int* __restrict__ queue_head, OrderShape o, int units) {
+  extern __shared__ int hist[];
+  __shared__ int warp_sum[kOrderThreads / 32];
+  if (!*valid) return;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nbins = o.kvb * o.nbk;
+  for (int i = tid; i < nbins; i += kOrderThreads) hist[i] = 0;
+  if (tid == 0) *queue_head = 0;
+  __syncthreads();
+  for (int i = tid; i < o.n_items; i += kOrderThreads)
+    atomicAdd(&hist[order_bin(p, o, row_ptr, i, units)], 1);
+  __syncthreads();
+  // exclusive scan of the histogram: a contiguous chunk per thread, then across the CTA
+  const int per = (nbins + kOrderThreads - 1) / kOrderThreads;
+  const int lo = min(nbins, tid * per), hi = min(nbins, lo + per);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += hist[i];
+  int x = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, d);
+    if (lane >= d) x += y;
+  }
+  if (lane == 31) warp_sum[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int v = warp_sum[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, d);
+      if (lane >= d) v += y;
+    }
+    warp_sum[lane] = v;
+  }
+  __syncthreads();
+  int run = x - sum + (wid > 0 ? warp_sum[wid - 1] : 0);
+  for (int i = lo; i < hi; ++i) {
+    const int c = hist[i];
+    hist[i] = run;
+    run += c;
+  }
+  __syncthreads();
+  for (int i = tid; i < o.n_items; i += kOrderThreads)
+    order[atomicAdd(&hist[order_bin(p, o, row_ptr, i, units)], 1)] = i;
+}
+
+cudaError_t launch_order(const ProblemDesc& p, int nb_max, SeqTables t, const int32_t* row_ptr,
+                         int32_t* order, int* queue_head, bool units, cudaStream_t s) {
+  const OrderShape o = order_shape(p, nb_max, units);
+  if (o.n_items == 0) return cudaSuccess;
+  const size_t smem = sizeof(int) * static_cast<size_t>(o.kvb) * o.nbk;
+  cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  order_kernel<<<1, kOrderThreads, smem, s>>>(p, t.valid, row_ptr, order, queue_head, o,
+                                              units ? 1 : 0);
   return cudaGetLastError();
 }
 

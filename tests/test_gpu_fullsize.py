@@ -20,15 +20,23 @@ import parity as PT
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    ("tiny_fp32_n2048", None),
-    ("llama8b_bf16_n8192", None),
-    ("llama8b_bf16_n32768", 0.0),
-    ("llama8b_bf16_n32768", 0.05),
-    ("llama8b_bf16_n32768", 0.1),
-    ("llama8b_bf16_n32768", 0.2),
-    ("llama8b_bf16_n131072", None),
-    ("llama8b_e4m3_n131072", None),
-    ("varlen8_bf16_t264192", None),
+    ("tiny_fp32_n2048", None, 1.0),
+    ("llama8b_bf16_n8192", None, 1.0),
+    ("llama8b_bf16_n32768", 0.0, 1.0),
+    ("llama8b_bf16_n32768", 0.05, 1.0),
+    ("llama8b_bf16_n32768", 0.1, 1.0),
+    ("llama8b_bf16_n32768", 0.2, 1.0),
+    ("llama8b_bf16_n131072", None, 1.0),
+    ("llama8b_e4m3_n131072", None, 1.0),
+    ("varlen8_bf16_t264192", None, 1.0),
+    # The sparse regime (labelled supplementary workloads): the same layers with Q multiplied by
+    # q_gain, which widens the pooled-score spread the way trained models' larger logits do; at
+    # alpha = 0.1 the 131072-token layer then keeps about 50 %, 20 % and 5 % of its causal blocks.
+    ("llama8b_bf16_n131072", None, 290.0),
+    ("llama8b_bf16_n131072", None, 340.0),
+    ("llama8b_bf16_n131072", None, 415.0),
+    ("llama8b_e4m3_n131072", None, 340.0),
+    ("varlen8_bf16_t264192", None, 340.0),
 ]
 
 
@@ -53,9 +61,10 @@ def sample_blocks(w, cu, rng):
     return sorted(set(picks)), lay
 
 
-@pytest.mark.parametrize("name,alpha", CASES, ids=[f"{n}-a{a}" for n, a in CASES])
-def test_full_size_parity(name, alpha):
-    w = WORKLOADS[name]
+@pytest.mark.parametrize("name,alpha,q_gain", CASES,
+                         ids=[f"{n}-a{a}-g{g:g}" for n, a, g in CASES])
+def test_full_size_parity(name, alpha, q_gain):
+    w = WORKLOADS[name].with_(q_gain=q_gain)
     if alpha is not None:
         w = w.with_(alpha=alpha)
     data = generate(w, workers=default_workers())
@@ -101,5 +110,8 @@ def test_full_size_parity(name, alpha):
                                              torch.from_numpy(np.concatenate(l_g)),
                                              np.concatenate(o_r), np.concatenate(l_r), w.dtype)
     density = len(ora_ci) / (w.hq * O.total_pairs(cu, w.block))
-    print(f"{name} alpha={w.alpha}: density={density:.4f} near-threshold={n_near} "
-          f"sampled blocks={len(picks)} O max/mean err={err_max:.2e}/{err_mean:.2e}")
+    if q_gain > 1.0:  # the supplementary workloads must really be sparse
+        assert density < 0.75, density
+    print(f"{name} alpha={w.alpha} q_gain={q_gain:g}: density={density:.4f} "
+          f"near-threshold={n_near} sampled blocks={len(picks)} "
+          f"O max/mean err={err_max:.2e}/{err_mean:.2e}")
