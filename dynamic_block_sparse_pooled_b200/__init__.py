@@ -32,7 +32,8 @@ EXPORTS = ("fpx_num_blocks", "fpx_scores_elems", "fpx_rows", "fpx_max_nnz", "fpx
            "fpx_select", "fpx_sparse_prefill", "fpx_attention_path", "fpx_select_noalloc",
            "fpx_select_noalloc_max_bytes", "fpx_diag_bounded_wait", "fpx_block_scores_paged",
            "fpx_sparse_prefill_paged", "fpx_block_scores_rescue", "fpx_select_rescue",
-           "fpx_diag_exp2")
+           "fpx_diag_exp2", "fpx_pattern_words", "fpx_vs_workspace_bytes", "fpx_probe_patterns",
+           "fpx_vs_select", "fpx_vs_prefill")
 
 
 class FpxError(RuntimeError):
@@ -108,6 +109,16 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fpx_diag_bounded_wait.restype = ctypes.c_int
     lib.fpx_diag_exp2.argtypes = [vp, vp, i64, vp]
     lib.fpx_diag_exp2.restype = ctypes.c_int
+    lib.fpx_pattern_words.argtypes = [P]
+    lib.fpx_pattern_words.restype = sz
+    lib.fpx_vs_workspace_bytes.argtypes = [P, i32]
+    lib.fpx_vs_workspace_bytes.restype = sz
+    lib.fpx_probe_patterns.argtypes = [P, vp, vp, i32, f32, f32, vp, vp, vp, sz, vp]
+    lib.fpx_probe_patterns.restype = ctypes.c_int
+    lib.fpx_vs_select.argtypes = [P, vp, vp, vp, vp, i64, vp, vp, sz, vp]
+    lib.fpx_vs_select.restype = ctypes.c_int
+    lib.fpx_vs_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fpx_vs_prefill.restype = ctypes.c_int
     K = ctypes.POINTER(PagedKV)
     lib.fpx_block_scores_paged.argtypes = [P, vp, vp, K, vp, vp, sz, vp]
     lib.fpx_block_scores_paged.restype = ctypes.c_int
@@ -360,3 +371,81 @@ def prefill(q, k, v, block: int, alpha: float, cu_seqlens=None, sink_blocks: int
     check(status(ws, stream), "device status")
     return dict(problem=pf, scores=scores, row_ptr=row_ptr, col_idx=col_idx, nnz=nnz, o=o,
                 lse=lse)
+
+
+# ---- query-probe vertical / slash path ------------------------------------------------------
+
+def pattern_words(pf: Prefill) -> int:
+    """uint32 words per head of the vertical / slash bitmasks (ceil(T / 32))."""
+    return load().fpx_pattern_words(pf.ptr)
+
+
+def vs_workspace(pf: Prefill, n_probe: int, device=None) -> torch.Tensor:
+    """A zeroed workspace for fpx_probe_patterns, fpx_vs_select and fpx_vs_prefill."""
+    n = load().fpx_vs_workspace_bytes(pf.ptr, int(n_probe))
+    if n == 0:
+        raise FpxError(-2, "fpx_vs_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def probe_patterns(pf: Prefill, q: torch.Tensor, k: torch.Tensor, n_probe: int, alpha_v: float,
+                   alpha_s: float, ws: torch.Tensor, vert=None, slash=None, stream=None):
+    """fpx_probe_patterns -> (vert_bits, slash_bits): int32 [Hq, words] holding the uint32
+    bitmasks (bit cu[s] + x of head h: key token / offset x of sequence s)."""
+    shape = (pf.struct.hq, max(1, pattern_words(pf)))
+    vert = torch.empty(shape, dtype=torch.int32, device=q.device) if vert is None else vert
+    slash = torch.empty(shape, dtype=torch.int32, device=q.device) if slash is None else slash
+    for t in (vert, slash):
+        if t.dtype != torch.int32 or t.numel() < shape[0] * shape[1] or not t.is_contiguous():
+            raise ValueError(f"bitmask must be a contiguous int32 tensor of {shape} words")
+    check(load().fpx_probe_patterns(pf.ptr, _ptr(q), _ptr(k), int(n_probe), float(alpha_v),
+                                    float(alpha_s), _ptr(vert), _ptr(slash), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "fpx_probe_patterns")
+    return vert, slash
+
+
+def vs_select(pf: Prefill, vert: torch.Tensor, slash: torch.Tensor, ws: torch.Tensor,
+              row_ptr=None, col_idx=None, nnz=None, capacity: Optional[int] = None, stream=None):
+    """fpx_vs_select -> (row_ptr, col_idx, nnz): key blocks that can hold an allowed key."""
+    dev = vert.device
+    if row_ptr is None:
+        row_ptr = torch.empty(pf.rows + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        cap = pf.struct.hq * pf.tri if capacity is None else capacity
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    cap = col_idx.numel() if capacity is None else capacity
+    if nnz is None:
+        nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    _check_csr_outputs(pf, row_ptr, col_idx, nnz, cap)
+    check(load().fpx_vs_select(pf.ptr, _ptr(vert), _ptr(slash), _ptr(row_ptr), _ptr(col_idx), cap,
+                               _ptr(nnz), _ptr(ws), ws.numel(), _stream(stream)), "fpx_vs_select")
+    return row_ptr, col_idx, nnz
+
+
+def vs_prefill(pf: Prefill, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+               vert: torch.Tensor, slash: torch.Tensor, row_ptr: torch.Tensor,
+               col_idx: torch.Tensor, ws: torch.Tensor, o=None, lse=None, stream=None):
+    """fpx_vs_prefill -> (O, LSE) under the vertical / slash token mask."""
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    check(load().fpx_vs_prefill(pf.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(vert), _ptr(slash),
+                                _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(lse), _ptr(ws),
+                                ws.numel(), _stream(stream)), "fpx_vs_prefill")
+    return o, lse
+
+
+def vs_path(q, k, v, block: int, n_probe: int, alpha_v: float, alpha_s: float, cu_seqlens=None,
+            softmax_scale: float = 0.0, q_scale=None, k_scale=None, v_scale=None,
+            stream=None) -> dict:
+    """The query-probe path on one stream: probes -> vertical / slash bitmasks -> candidate
+    blocks -> masked attention.  Raises on any recorded device-side error."""
+    pf = problem(q, k, block, cu_seqlens, softmax_scale, q_scale, k_scale, v_scale)
+    ws = vs_workspace(pf, n_probe, q.device)
+    vert, slash = probe_patterns(pf, q, k, n_probe, alpha_v, alpha_s, ws, stream=stream)
+    row_ptr, col_idx, nnz = vs_select(pf, vert, slash, ws, stream=stream)
+    o, lse = vs_prefill(pf, q, k, v, vert, slash, row_ptr, col_idx, ws, stream=stream)
+    check(status(ws, stream), "device status")
+    return dict(problem=pf, vert=vert, slash=slash, row_ptr=row_ptr, col_idx=col_idx, nnz=nnz,
+                o=o, lse=lse)

@@ -212,6 +212,58 @@ fpx_status fpx_select_rescue(const fpx_problem* p, const float* scores, const fl
                              size_t ws_bytes, fpx_stream_t stream);
 
 /*
+ * Query-probe vertical / slash pattern discovery (FlashPrefill §3 Method, "Instantaneous Pattern
+ * Discovery": uniformly distributed query probes find the vertical and slash patterns; §1
+ * Introduction names the three pattern types).  The page gives no formula; the library
+ * implements this reading, per sequence s of n tokens and Q head h:
+ *   probes   m = min(n_probe, n) query tokens at pos_p = ceil((p + 1) n / m) - 1, p < m;
+ *   A[p, j]  the exact causal softmax row of probe p: softmax over keys j <= pos_p of
+ *            scale * <q_pos_p, k_j> (dequantised values for e4m3);
+ *   Amax     max over p and j of A[p, j];
+ *   vertical key j   iff alpha_v == 0 or max_p A[p, j] >= alpha_v * Amax;
+ *   slash offset d   iff alpha_s == 0 or max_p A[p, pos_p - d] >= alpha_s * Amax
+ *   (the page's max-based threshold, applied to the probes' attention).
+ * Output, a token-granular index in bitmask form: vert_bits and slash_bits, device uint32
+ *   [hq * words] each with words = fpx_pattern_words(p) = ceil(T / 32); bit b of head h is word
+ *   h * words + b / 32, bit b % 32; bit cu[s] + x marks key token x (vert_bits) or offset x
+ *   (slash_bits) of sequence s.  Both arrays are overwritten (bits of other sequences included).
+ * Limits: bf16 or e4m3, d = 128, block = 128 (fpx_attention_path(p) == 1); 1 <= n_probe and
+ *   (hq / hkv) * n_probe <= 512, else FPX_ERR_UNSUPPORTED.  alpha_v, alpha_s >= 0 (NaN:
+ *   FPX_ERR_INVALID_ARG).
+ * ws: device workspace >= fpx_vs_workspace_bytes(p, n_probe) (serves all three entry points of
+ *   this path).
+ */
+size_t fpx_pattern_words(const fpx_problem* p);
+size_t fpx_vs_workspace_bytes(const fpx_problem* p, int32_t n_probe);
+fpx_status fpx_probe_patterns(const fpx_problem* p, const void* q, const void* k,
+                              int32_t n_probe, float alpha_v, float alpha_s, uint32_t* vert_bits,
+                              uint32_t* slash_bits, void* ws, size_t ws_bytes,
+                              fpx_stream_t stream);
+
+/*
+ * Key-block candidates of the vertical / slash attention: CSR (same layout and capacity rules as
+ * fpx_select) listing, for every row (h, s, I), the key blocks J <= I that can hold a key some
+ * query of block I attends: J holds a vertical of head h, or a slash offset of head h lies in
+ * [(I - J) B - B + 1, (I - J) B + B - 1].  Any bitmasks in the layout above are accepted.
+ */
+fpx_status fpx_vs_select(const fpx_problem* p, const uint32_t* vert_bits,
+                         const uint32_t* slash_bits, int32_t* row_ptr, int32_t* col_idx,
+                         int64_t col_capacity, int64_t* nnz_d, void* ws, size_t ws_bytes,
+                         fpx_stream_t stream);
+
+/*
+ * Exact attention under the vertical / slash token mask: query token i (local) of sequence s,
+ * Q head h attends key j <= i iff bit cu[s] + j of vert_bits[h] or bit cu[s] + (i - j) of
+ * slash_bits[h] is set, among the key blocks its CSR row (h, s, i / B) lists (a list from
+ * fpx_vs_select covers every such key).  O and LSE as fpx_sparse_prefill; a row that no key
+ * reaches gets O = 0 and LSE = -inf.  Tensor-core path only (fpx_attention_path(p) == 1).
+ */
+fpx_status fpx_vs_prefill(const fpx_problem* p, const void* q, const void* k, const void* v,
+                          const uint32_t* vert_bits, const uint32_t* slash_bits,
+                          const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
+                          void* ws, size_t ws_bytes, fpx_stream_t stream);
+
+/*
  * Allocation-free variant of fpx_select (the paper has no counterpart; it exists for callers).
  *   Some callers cannot allocate device memory where they run: a plugin whose host framework
  *   owns all device memory and offers no scratch buffer, or latency-critical code that must not
