@@ -393,6 +393,7 @@ def sub_records(fpx, args, device, sdpa_ms_128k):
         if sdpa_ms_128k:
             r["speedup_vs_sdpa_dense"] = round(sdpa_ms_128k / r["attn_ms"], 3)
         out["sparse"].append(r)
+    out["patterns"] = pattern_record(fpx, f32, device, steps)
     del f32
     for name, alphas in (("llama8b_bf16_n32768", (0.0, 0.05, 0.1, 0.2)),
                          ("llama8b_e4m3_n131072", (None,)), ("varlen8_bf16_t264192", (None,))):
@@ -407,6 +408,53 @@ def sub_records(fpx, args, device, sdpa_ms_128k):
             out["configs"].append({"workload": w.name, "alpha": w.alpha, **r})
         del data
     return out
+
+
+def pattern_record(fpx, f32, device, steps, gain=40.0, n_probe=64, alpha_v=0.01, alpha_s=0.01):
+    """The query-probe vertical / slash path on the 131072-token layer (Q x q_gain): probe
+    discovery, candidate blocks and the token-masked attention, each timed with CUDA events
+    (3 warm-up calls, then `steps`), with the sizes of what the probes selected."""
+    try:
+        w = WORKLOADS["llama8b_bf16_n131072"].with_(q_gain=gain)
+        q = (f32["q"] * np.float32(gain)).to(torch.bfloat16).to(device)
+        k = f32["k"].to(torch.bfloat16).to(device)
+        v = f32["v"].to(torch.bfloat16).to(device)
+        cu = f32["cu_seqlens"]
+        pf = fpx.problem(q, k, w.block, cu)
+        ws = fpx.vs_workspace(pf, n_probe, device)
+        vert, slash = fpx.probe_patterns(pf, q, k, n_probe, alpha_v, alpha_s, ws)
+        rp, ci, nnz = fpx.vs_select(pf, vert, slash, ws)
+        o, lse = fpx.vs_prefill(pf, q, k, v, vert, slash, rp, ci, ws)
+        stages = {
+            "probe_ms": lambda: fpx.probe_patterns(pf, q, k, n_probe, alpha_v, alpha_s, ws,
+                                                   vert=vert, slash=slash),
+            "select_ms": lambda: fpx.vs_select(pf, vert, slash, ws, row_ptr=rp, col_idx=ci,
+                                               nnz=nnz),
+            "attn_ms": lambda: fpx.vs_prefill(pf, q, k, v, vert, slash, rp, ci, ws, o=o, lse=lse),
+        }
+        res = {"workload": w.name, "q_gain": gain, "n_probe": n_probe, "alpha_v": alpha_v,
+               "alpha_s": alpha_s}
+        for name, fn in stages.items():
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize(device)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(steps):
+                fn()
+            b.record()
+            torch.cuda.synchronize(device)
+            res[name] = round(a.elapsed_time(b) / steps, 4)
+        if fpx.status(ws) != 0:
+            return {"unavailable": f"device status {fpx.status(ws)}"}
+        bits = lambda t: int(np.unpackbits(t.cpu().numpy().view(np.uint8)).sum())  # noqa: E731
+        res["verticals"] = bits(vert)
+        res["slashes"] = bits(slash)
+        res["candidate_density"] = round(int(nnz.item()) / (w.hq * pairs(w)), 6)
+        res["dense_equiv_tflops"] = round(dense_flops(w) / (res["attn_ms"] * 1e-3) / 1e12, 1)
+        return res
+    except Exception as e:  # reported, never hidden
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
 
 
 def run_ours(args, rank, world, device):

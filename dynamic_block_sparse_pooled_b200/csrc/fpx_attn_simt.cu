@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
     ProblemDesc p, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx, OT* __restrict__ o,
     float* __restrict__ lse, SeqTables t, const int32_t* __restrict__ order, StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   constexpr int TPR = D / 64;  // threads per query row
   __shared__ float sk[kSimtChunk][D + 1];
   __shared__ float sv[kSimtChunk][D + 1];
@@ -142,13 +143,13 @@ static cudaError_t launch_simt_t(const ProblemDesc& p, const void* q, const void
   const int R = p.hq * p.nb_total;
   const int threads = p.block * (p.d / 64);
   if (p.d == 128)
-    attn_simt_kernel<T, OT, 128><<<R, threads, 0, s>>>(
-        p, static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), row_ptr,
-        col_idx, static_cast<OT*>(o), lse, t, order, st);
+    FPX_CHAIN((attn_simt_kernel<T, OT, 128>), R, threads, 0, s, p, static_cast<const T*>(q),
+              static_cast<const T*>(k), static_cast<const T*>(v), row_ptr, col_idx,
+              static_cast<OT*>(o), lse, t, order, st);
   else
-    attn_simt_kernel<T, OT, 64><<<R, threads, 0, s>>>(
-        p, static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), row_ptr,
-        col_idx, static_cast<OT*>(o), lse, t, order, st);
+    FPX_CHAIN((attn_simt_kernel<T, OT, 64>), R, threads, 0, s, p, static_cast<const T*>(q),
+              static_cast<const T*>(k), static_cast<const T*>(v), row_ptr, col_idx,
+              static_cast<OT*>(o), lse, t, order, st);
   return cudaGetLastError();
 }
 

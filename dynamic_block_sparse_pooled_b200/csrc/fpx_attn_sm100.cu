@@ -251,6 +251,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const int32_t* __restrict__ order, int* __restrict__ queue_head, int n_units,
                const uint32_t* __restrict__ vbits, const uint32_t* __restrict__ sbits, int words,
                StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   using C = Cfg<kFp8>;
   constexpr unsigned kFull = 0xffffffffu;
   if (!*tab.valid) return;  // inconsistent cu_seqlens (recorded by the plan kernel)
@@ -847,9 +848,9 @@ cudaError_t launch_attn_tc(const ProblemDesc& p, fpx_dtype dt, const void* q, co
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM takes units from the queue (heaviest first) until it is empty
   const int64_t grid = units < sm_count() ? units : sm_count();
-  kern<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(
-      mq, mk, mv, p, row_ptr, col_idx, static_cast<__nv_bfloat16*>(o), lse, t, order, queue_head,
-      static_cast<int>(units), vbits, sbits, words, st);
+  FPX_CHAIN(kern, static_cast<unsigned>(grid), kThreads, kSmemBytes, s, mq, mk, mv, p, row_ptr,
+            col_idx, static_cast<__nv_bfloat16*>(o), lse, t, order, queue_head,
+            static_cast<int>(units), vbits, sbits, words, st);
   return cudaGetLastError();
 }
 

@@ -124,6 +124,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  Every library kernel is launched with programmatic stream
+// serialization (launch_chained) and starts with pdl_enter(): it waits until the kernel before it
+// on the stream has completed and its writes are visible (griddepcontrol.wait), then lets the
+// kernel after it be scheduled (launch_dependents), so that kernel's launch and CTA set-up overlap
+// this one's execution instead of following its end.  Without the launch attribute both
+// instructions are no-ops.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Upper bound for any single device-side wait.  A correct schedule waits microseconds; the
 // bound only turns a broken pipeline into FPX_ERR_TIMEOUT instead of a hung GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s

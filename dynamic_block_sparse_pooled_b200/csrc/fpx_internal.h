@@ -8,6 +8,33 @@
 
 namespace fpx {
 
+// Launches kern<<<grid, block, smem, s>>>(args...) with programmatic stream serialization (the
+// kernel calls pdl_enter() before it touches anything the previous kernel writes).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// launch_chained in a function returning cudaError_t: returns the error of a failed launch.
+// (A kernel name with template arguments is passed in parentheses.)
+#define FPX_CHAIN(kern, grid, block, smem, stream, ...)                                        \
+  do {                                                                                          \
+    const cudaError_t fpx_chain_err_ =                                                          \
+        ::fpx::launch_chained(kern, dim3(grid), dim3(block), smem, stream, __VA_ARGS__);       \
+    if (fpx_chain_err_ != cudaSuccess) return fpx_chain_err_;                                   \
+  } while (0)
+
 // Stage 0 building block, shared by all entry points: per-sequence tables + cu_seqlens checks.
 cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cudaStream_t s);
 

@@ -103,6 +103,7 @@ __device__ __forceinline__ int seq_of_chunk(const int32_t* chunk_base, int num_s
 __global__ void __launch_bounds__(1024) probe_plan_kernel(ProblemDesc p, SeqTables t,
                                                           int chunk_blocks,
                                                           int32_t* __restrict__ chunk_base) {
+  pdl_enter();  // after the previous kernel on the stream
   __shared__ int warp_sum[32];
   if (!*t.valid) return;
   const int S = p.num_seqs, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -161,6 +162,7 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
                   const int32_t* __restrict__ chunk_base, float2* __restrict__ partial,
                   const float2* __restrict__ bound, uint32_t* __restrict__ vbits,
                   uint32_t* __restrict__ sbits, StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   using C = PCfg<kFp8>;
   constexpr int kRowThreads = kTiles * 128;
   constexpr int kCtrlWarp = kTiles * 4;
@@ -384,6 +386,7 @@ __global__ void __launch_bounds__(512) probe_reduce_kernel(
     ProblemDesc p, ProbeArgs a, SeqTables tab, const int32_t* __restrict__ chunk_base,
     const float2* __restrict__ partial, float2* __restrict__ bound, uint32_t* __restrict__ vbits,
     uint32_t* __restrict__ sbits) {
+  pdl_enter();  // after the previous kernel on the stream
   __shared__ float warp_max[16];
   if (!*tab.valid) return;
   const int s = blockIdx.x, h = blockIdx.y;
@@ -459,6 +462,7 @@ __global__ void vs_flags_kernel(ProblemDesc p, SeqTables tab, int words,
                                 const uint32_t* __restrict__ vbits,
                                 const uint32_t* __restrict__ sbits, uint8_t* __restrict__ vflag,
                                 uint8_t* __restrict__ sflag) {
+  pdl_enter();  // after the previous kernel on the stream
   if (!*tab.valid) return;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= static_cast<int64_t>(p.hq) * p.nb_total) return;
@@ -489,6 +493,7 @@ __global__ void __launch_bounds__(kVsWarps * 32) vs_count_kernel(
     ProblemDesc p, SeqTables tab, const uint8_t* __restrict__ vflag,
     const uint8_t* __restrict__ sflag, int32_t* __restrict__ counts,
     int64_t* __restrict__ cta_tot, uint32_t* __restrict__ mask, int mask_words) {
+  pdl_enter();  // after the previous kernel on the stream
   __shared__ int w_tot[kVsWarps];
   if (!*tab.valid) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -541,8 +546,8 @@ static cudaError_t launch_pass_t(const CUtensorMap& mk, const ProblemDesc& p,
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<dim3(total_chunks, p.hkv), kTiles * 128 + 32, smem, s>>>(
-      mk, p, a, static_cast<const uint8_t*>(q), t, chunk_base, partial, bound, vb, sb, st);
+  FPX_CHAIN(kern, dim3(total_chunks, p.hkv), kTiles * 128 + 32, smem, s, mk, p, a,
+            static_cast<const uint8_t*>(q), t, chunk_base, partial, bound, vb, sb, st);
   return cudaGetLastError();
 }
 
@@ -584,7 +589,7 @@ cudaError_t launch_probe(const ProblemDesc& p, fpx_dtype dt, const void* q, cons
   cudaError_t e = cudaMemsetAsync(vbits, 0, bytes, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(sbits, 0, bytes, s);
   if (e != cudaSuccess || p.nb_total == 0) return e;
-  probe::probe_plan_kernel<<<1, 1024, 0, s>>>(p, t, chunk_blocks, chunk_base);
+  FPX_CHAIN(probe::probe_plan_kernel, 1, 1024, 0, s, p, t, chunk_blocks, chunk_base);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   CUtensorMap mk;
   if (!make_tmap_rows128(&mk, k, p.total_tokens, p.hkv, p.d, fp8 ? 1 : 2)) {
@@ -594,8 +599,8 @@ cudaError_t launch_probe(const ProblemDesc& p, fpx_dtype dt, const void* q, cons
   if ((e = launch_pass<false>(mk, p, fp8, a, q, t, chunk_base, total_chunks, partial, nullptr,
                               vbits, sbits, st, s)) != cudaSuccess)
     return e;
-  probe::probe_reduce_kernel<<<dim3(p.num_seqs, p.hq), 512, 0, s>>>(p, a, t, chunk_base, partial,
-                                                                    bound, vbits, sbits);
+  FPX_CHAIN(probe::probe_reduce_kernel, dim3(p.num_seqs, p.hq), 512, 0, s, p, a, t, chunk_base,
+            partial, bound, vbits, sbits);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.all_v && a.all_s) return cudaSuccess;
   return launch_pass<true>(mk, p, fp8, a, q, t, chunk_base, total_chunks, partial, bound, vbits,
@@ -608,13 +613,13 @@ cudaError_t launch_vs_count(const ProblemDesc& p, SeqTables t, const uint32_t* v
                             cudaStream_t s) {
   const int64_t R = static_cast<int64_t>(p.hq) * p.nb_total;
   if (R == 0) return cudaSuccess;
-  probe::vs_flags_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, s>>>(
-      p, t, words, vbits, sbits, vflag, sflag);
+  FPX_CHAIN(probe::vs_flags_kernel, static_cast<unsigned>((R + 255) / 256), 256, 0, s, p, t, words,
+            vbits, sbits, vflag, sflag);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  probe::vs_count_kernel<<<static_cast<unsigned>((R + probe::kVsWarps - 1) / probe::kVsWarps),
-                           probe::kVsWarps * 32, 0, s>>>(p, t, vflag, sflag, counts, cta_tot, mask,
-                                                        mask_words);
+  FPX_CHAIN(probe::vs_count_kernel,
+            static_cast<unsigned>((R + probe::kVsWarps - 1) / probe::kVsWarps),
+            probe::kVsWarps * 32, 0, s, p, t, vflag, sflag, counts, cta_tot, mask, mask_words);
   return cudaGetLastError();
 }
 

@@ -55,6 +55,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant_
                 ProblemDesc p, float* __restrict__ scores, const int32_t* __restrict__ blk_base,
                 const int64_t* __restrict__ tri_base, const int32_t* __restrict__ valid,
                 StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   // lower-triangle tile index -> (x, y), y <= x
   const int kt = blockIdx.x;
   int x = static_cast<int>((sqrtf(8.f * kt + 1.f) - 1.f) * 0.5f);
@@ -252,8 +253,8 @@ cudaError_t launch_score_tc(const ProblemDesc& p, const float* qhi, const float*
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSSmemBytes));
   if (e != cudaSuccess) return e;
-  score_tc_kernel<<<grid, kSThreads, kSSmemBytes, s>>>(mqh, mql, mkh, mkl, p, scores, t.blk_base,
-                                                        t.tri_base, t.valid, st);
+  FPX_CHAIN(score_tc_kernel, grid, kSThreads, kSSmemBytes, s, mqh, mql, mkh, mkl, p, scores,
+            t.blk_base, t.tri_base, t.valid, st);
   return cudaGetLastError();
 }
 

@@ -32,6 +32,7 @@ constexpr int kPlanThreads = 256;
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(ProblemDesc p, SeqTables t,
                                                             StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   __shared__ int64_t w_nb[kPlanThreads / 32], w_tri[kPlanThreads / 32];
   __shared__ int s_bad;
   const int S = p.num_seqs;
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(ProblemDesc p, SeqTa
 }
 
 cudaError_t launch_plan(const ProblemDesc& p, SeqTables t, StatusBlock* st, cudaStream_t s) {
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(p, t, st);
+  FPX_CHAIN(plan_kernel, 1, kPlanThreads, 0, s, p, t, st);
   return cudaGetLastError();
 }
 
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(ProblemDesc p, const
                                                             const int32_t* __restrict__ blk_base,
                                                             const int32_t* __restrict__ valid,
                                                             int q_chunks, StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   constexpr int V = Vec16<T>::N;
   if (!*valid) return;
   const int b = blockIdx.x;
@@ -251,19 +253,19 @@ cudaError_t launch_pool(const ProblemDesc& p, fpx_dtype dt, const void* q, const
   dim3 grid(p.nb_total, q_chunks + k_chunks);
   switch (dt) {
     case FPX_F32:
-      pool_kernel<float><<<grid, kPoolThreads, 0, s>>>(p, static_cast<const float*>(q),
-                                                        static_cast<const float*>(k), qbar, kbar,
-                                                        qlo, klo, blk_base, t.valid, q_chunks, st);
+      FPX_CHAIN(pool_kernel<float>, grid, kPoolThreads, 0, s, p, static_cast<const float*>(q),
+                static_cast<const float*>(k), qbar, kbar, qlo, klo, blk_base, t.valid, q_chunks,
+                st);
       break;
     case FPX_BF16:
-      pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, s>>>(
-          p, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar,
-          kbar, qlo, klo, blk_base, t.valid, q_chunks, st);
+      FPX_CHAIN(pool_kernel<__nv_bfloat16>, grid, kPoolThreads, 0, s, p,
+                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar,
+                kbar, qlo, klo, blk_base, t.valid, q_chunks, st);
       break;
     default:
-      pool_kernel<__nv_fp8_e4m3><<<grid, kPoolThreads, 0, s>>>(
-          p, static_cast<const __nv_fp8_e4m3*>(q), static_cast<const __nv_fp8_e4m3*>(k), qbar,
-          kbar, qlo, klo, blk_base, t.valid, q_chunks, st);
+      FPX_CHAIN(pool_kernel<__nv_fp8_e4m3>, grid, kPoolThreads, 0, s, p,
+                static_cast<const __nv_fp8_e4m3*>(q), static_cast<const __nv_fp8_e4m3*>(k), qbar,
+                kbar, qlo, klo, blk_base, t.valid, q_chunks, st);
       break;
   }
   return cudaGetLastError();
@@ -289,6 +291,7 @@ __global__ void __launch_bounds__(kRadWarps * 32) radius_kernel(
     const float* __restrict__ kbar, const float* __restrict__ qlo, const float* __restrict__ klo,
     float* __restrict__ qnorm, float* __restrict__ radius, const int32_t* __restrict__ blk_base,
     const int32_t* __restrict__ valid) {
+  pdl_enter();  // after the previous kernel on the stream
   constexpr int E = D / 32;  // elements per lane
   if (!*valid) return;
   const int lane = threadIdx.x & 31;
@@ -362,9 +365,8 @@ cudaError_t launch_radius(const ProblemDesc& p, fpx_dtype dt, const void* k, con
   const int64_t pairs = static_cast<int64_t>(p.nb_total) * (p.hkv + p.hq);
   const unsigned grid = static_cast<unsigned>((pairs + kRadWarps - 1) / kRadWarps);
 #define FPX_RAD(T, DD)                                                                        \
-  radius_kernel<T, DD><<<grid, kRadWarps * 32, 0, s>>>(p, static_cast<const T*>(k), qbar, kbar, \
-                                                       qlo, klo, qnorm, radius, t.blk_base,   \
-                                                       t.valid)
+  FPX_CHAIN((radius_kernel<T, DD>), grid, kRadWarps * 32, 0, s, p, static_cast<const T*>(k),   \
+            qbar, kbar, qlo, klo, qnorm, radius, t.blk_base, t.valid)
   if (p.d == 128) {
     if (dt == FPX_F32) FPX_RAD(float, 128);
     else if (dt == FPX_BF16) FPX_RAD(__nv_bfloat16, 128);
@@ -394,6 +396,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ProblemDesc p,
                                                               const int32_t* __restrict__ blk_base,
                                                               const int64_t* __restrict__ tri_base,
                                                               const int32_t* __restrict__ valid) {
+  pdl_enter();  // after the previous kernel on the stream
   if (!*valid) return;
   extern __shared__ float4 score_smem[];
   float* sq = reinterpret_cast<float*>(score_smem);  // [D][64] (transposed)
@@ -477,11 +480,11 @@ cudaError_t launch_score(const ProblemDesc& p, fpx_dtype, const float* qbar, con
   if (p.d == 128) {
     cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    score_kernel<128><<<grid, kScoreThreads, smem, s>>>(p, qbar, kbar, scores, t.blk_base,
-                                                         t.tri_base, t.valid);
+    FPX_CHAIN(score_kernel<128>, grid, kScoreThreads, smem, s, p, qbar, kbar, scores, t.blk_base,
+              t.tri_base, t.valid);
   } else {
-    score_kernel<64><<<grid, kScoreThreads, smem, s>>>(p, qbar, kbar, scores, t.blk_base,
-                                                        t.tri_base, t.valid);
+    FPX_CHAIN(score_kernel<64>, grid, kScoreThreads, smem, s, p, qbar, kbar, scores, t.blk_base,
+              t.tri_base, t.valid);
   }
   return cudaGetLastError();
 }
@@ -544,6 +547,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_count_kernel(
     float* __restrict__ rowmax, int32_t* __restrict__ counts, int64_t* __restrict__ cta_tot,
     uint32_t* __restrict__ mask, int mask_words, const float* __restrict__ qn,
     const float* __restrict__ rad, float alpha_r, SeqTables t) {
+  pdl_enter();  // after the previous kernel on the stream
   if (!*t.valid) return;
   __shared__ int w_tot[kSelWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -625,6 +629,7 @@ __global__ void __launch_bounds__(kScanThreads) select_scan_kernel(
     int R, int nblk, int64_t* __restrict__ cta_tot, int32_t* __restrict__ row_ptr,
     int64_t capacity, int64_t* __restrict__ nnz_d, int* __restrict__ overflow,
     const int32_t* __restrict__ valid, StatusBlock* st) {
+  pdl_enter();  // after the previous kernel on the stream
   __shared__ int64_t warp_tot[32];
   if (!*valid) {  // inconsistent cu_seqlens (already recorded): publish an empty CSR
     for (int i = threadIdx.x; i <= R; i += blockDim.x) row_ptr[i] = 0;
@@ -689,6 +694,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_emit_kernel(
     int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
     const int* __restrict__ overflow, const uint32_t* __restrict__ mask, int mask_words,
     SeqTables t) {
+  pdl_enter();  // after the previous kernel on the stream
   if (!*t.valid || *overflow) return;  // the scan published an empty CSR
   __shared__ int32_t s_off[kSelRows];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -738,12 +744,12 @@ cudaError_t launch_select_finish(const ProblemDesc& p, int32_t* row_ptr, int32_t
                                  int mask_words, SeqTables t, StatusBlock* st, cudaStream_t s) {
   const int R = p.hq * p.nb_total;
   const int nblk = select_ctas(p);
-  select_scan_kernel<<<1, kScanThreads, 0, s>>>(R, nblk, cta_tot, row_ptr, capacity, nnz_d,
-                                                overflow, t.valid, st);
+  FPX_CHAIN(select_scan_kernel, 1, kScanThreads, 0, s, R, nblk, cta_tot, row_ptr, capacity, nnz_d,
+            overflow, t.valid, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || R == 0) return e;
-  select_emit_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, counts, cta_tot, row_ptr, col_idx,
-                                                     overflow, mask, mask_words, t);
+  FPX_CHAIN(select_emit_kernel, nblk, kSelWarps * 32, 0, s, p, counts, cta_tot, row_ptr, col_idx,
+            overflow, mask, mask_words, t);
   return cudaGetLastError();
 }
 
@@ -756,18 +762,17 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
   const int R = p.hq * p.nb_total;
   const int nblk = select_ctas(p);
   if (R > 0) {
-    select_count_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, scores, alpha, sink, window, rowmax,
-                                                       counts, cta_tot, mask, mask_words, qn,
-                                                       rad, alpha_r, t);
+    FPX_CHAIN(select_count_kernel, nblk, kSelWarps * 32, 0, s, p, scores, alpha, sink, window,
+              rowmax, counts, cta_tot, mask, mask_words, qn, rad, alpha_r, t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  select_scan_kernel<<<1, kScanThreads, 0, s>>>(R, nblk, cta_tot, row_ptr, capacity, nnz_d,
-                                                overflow, t.valid, st);
+  FPX_CHAIN(select_scan_kernel, 1, kScanThreads, 0, s, R, nblk, cta_tot, row_ptr, capacity, nnz_d,
+            overflow, t.valid, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || R == 0) return e;
-  select_emit_kernel<<<nblk, kSelWarps * 32, 0, s>>>(p, counts, cta_tot, row_ptr, col_idx,
-                                                     overflow, mask, mask_words, t);
+  FPX_CHAIN(select_emit_kernel, nblk, kSelWarps * 32, 0, s, p, counts, cta_tot, row_ptr, col_idx,
+            overflow, mask, mask_words, t);
   return cudaGetLastError();
 }
 
@@ -831,6 +836,7 @@ __device__ __forceinline__ int order_bin(const ProblemDesc& p, const OrderShape&
 __global__ void __launch_bounds__(kOrderThreads) order_kernel(
     ProblemDesc p, const int32_t* __restrict__ valid, const int32_t* __restrict__ row_ptr,
     int32_t* __restrict__ order, int* __restrict__ queue_head, OrderShape o, int units) {
+  pdl_enter();  // after the previous kernel on the stream
   extern __shared__ int hist[];
   __shared__ int warp_sum[kOrderThreads / 32];
   if (!*valid) return;
@@ -884,8 +890,8 @@ cudaError_t launch_order(const ProblemDesc& p, int nb_max, SeqTables t, const in
   cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  order_kernel<<<1, kOrderThreads, smem, s>>>(p, t.valid, row_ptr, order, queue_head, o,
-                                              units ? 1 : 0);
+  FPX_CHAIN(order_kernel, 1, kOrderThreads, smem, s, p, t.valid, row_ptr, order, queue_head, o,
+            units ? 1 : 0);
   return cudaGetLastError();
 }
 
