@@ -45,11 +45,9 @@ KERNELS_PER_STEP = 10  # plan+pool+score, plan+count+scan+emit, plan+order+atten
 ATTN_SOURCES = ("dynamic_block_sparse_pooled_b200/csrc/fpx_attn_sm100.cu",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_sm100.cuh",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_common.cuh")
-ATTN_TRAFFIC_DIGEST = "6658f110d9bd4973b8588fda2b31b76420b79e51a7fcadb43921af89dcf8db0b"
+ATTN_TRAFFIC_DIGEST = "6b793b6fb7ca1753bdc8ad6f8cb0608a19ff208e02c1a225b10169018174f519"
 ATTN_TRAFFIC = {
-    "llama8b_bf16_n131072": 3192360704 + 1084167168,
-    "llama8b_e4m3_n131072": 1204427264 + 1049897728,
-    "llama8b_bf16_n32768": 407483136 + 238002176,
+    "llama8b_bf16_n131072": 3303332864 + 1180280320,
 }
 
 
