@@ -789,6 +789,7 @@ cudaError_t launch_select(const ProblemDesc& p, const float* scores, float alpha
 // ------------------------------------------------------------------------------------------
 constexpr int kOrderThreads = 1024;
 constexpr int kOrderMaxBins = 16384;  // 64 KB of shared-memory histogram
+constexpr size_t kOrderSmemBudget = 200 * 1024;  // histogram + cached bins
 
 struct OrderShape {
   int slots, per_kv, n_items, nbk, cost_cap, kvb;  // kvb: KV-head groups (<= kOrderMaxBins)
@@ -835,18 +836,33 @@ __device__ __forceinline__ int order_bin(const ProblemDesc& p, const OrderShape&
 
 __global__ void __launch_bounds__(kOrderThreads) order_kernel(
     ProblemDesc p, const int32_t* __restrict__ valid, const int32_t* __restrict__ row_ptr,
-    int32_t* __restrict__ order, int* __restrict__ queue_head, OrderShape o, int units) {
+    int32_t* __restrict__ order, int* __restrict__ queue_head, OrderShape o, int units,
+    int cache_bins) {
   pdl_enter();  // after the previous kernel on the stream
-  extern __shared__ int hist[];
+  extern __shared__ int hist[];  // [kvb * nbk] counts, then (cache_bins) uint16 bin per item
   __shared__ int warp_sum[kOrderThreads / 32];
   if (!*valid) return;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int nbins = o.kvb * o.nbk;
+  uint16_t* bin_of = reinterpret_cast<uint16_t*>(hist + nbins);
   for (int i = tid; i < nbins; i += kOrderThreads) hist[i] = 0;
   if (tid == 0) *queue_head = 0;
   __syncthreads();
-  for (int i = tid; i < o.n_items; i += kOrderThreads)
-    atomicAdd(&hist[order_bin(p, o, row_ptr, i, units)], 1);
+  // pass 1: four items per thread in flight (their row_ptr loads are independent)
+  for (int i0 = tid; i0 < o.n_items; i0 += 4 * kOrderThreads) {
+    int bins[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kOrderThreads;
+      bins[u] = i < o.n_items ? order_bin(p, o, row_ptr, i, units) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (bins[u] < 0) continue;
+      atomicAdd(&hist[bins[u]], 1);
+      if (cache_bins) bin_of[i0 + u * kOrderThreads] = static_cast<uint16_t>(bins[u]);
+    }
+  }
   __syncthreads();
   // exclusive scan of the histogram: a contiguous chunk per thread, then across the CTA
   const int per = (nbins + kOrderThreads - 1) / kOrderThreads;
@@ -878,20 +894,27 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(
     run += c;
   }
   __syncthreads();
-  for (int i = tid; i < o.n_items; i += kOrderThreads)
-    order[atomicAdd(&hist[order_bin(p, o, row_ptr, i, units)], 1)] = i;
+  // pass 2: scatter (bins from shared memory, or recomputed when they did not fit)
+  for (int i = tid; i < o.n_items; i += kOrderThreads) {
+    const int bin = cache_bins ? static_cast<int>(bin_of[i]) : order_bin(p, o, row_ptr, i, units);
+    order[atomicAdd(&hist[bin], 1)] = i;
+  }
 }
 
 cudaError_t launch_order(const ProblemDesc& p, int nb_max, SeqTables t, const int32_t* row_ptr,
                          int32_t* order, int* queue_head, bool units, cudaStream_t s) {
   const OrderShape o = order_shape(p, nb_max, units);
   if (o.n_items == 0) return cudaSuccess;
-  const size_t smem = sizeof(int) * static_cast<size_t>(o.kvb) * o.nbk;
+  // the histogram, and the items' bins (uint16) when they fit in the shared memory budget
+  const size_t hist_bytes = sizeof(int) * static_cast<size_t>(o.kvb) * o.nbk;
+  const size_t bins_bytes = sizeof(uint16_t) * static_cast<size_t>(o.n_items);
+  const int cache_bins = hist_bytes + bins_bytes <= kOrderSmemBudget ? 1 : 0;
+  const size_t smem = hist_bytes + (cache_bins ? bins_bytes : 0);
   cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   FPX_CHAIN(order_kernel, 1, kOrderThreads, smem, s, p, t.valid, row_ptr, order, queue_head, o,
-            units ? 1 : 0);
+            units ? 1 : 0, cache_bins);
   return cudaGetLastError();
 }
 
