@@ -332,8 +332,8 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
           if (lane == 0) mbar_arrive(bar(kPSFree));  // S may be overwritten by the next block
         }
         const int nv = min(64, nvis - half * 64);  // visible columns of this half
-        if (nv <= 0) continue;
         if (!kMark) {
+          if (nv <= 0) continue;
           float mx = -CUDART_INF_F;
 #pragma unroll
           for (int j = 0; j < 64; ++j)
@@ -346,20 +346,46 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
           lrun = lrun * ex2_approx(mrun - mnew) + sum;  // mrun = -inf: 0 * 0
           mrun = mnew;
         } else {
+          // Marks, gathered before the atomics.  Verticals: the key column is the same for
+          // every lane, so a vote per column among the lanes of one Q head (a warp holds the
+          // probe rows of several heads when n_probe is not a multiple of 32) collects that
+          // head's hits, and its first lane sets them with one atomicOr per 32-bit word.
+          // Slashes: a lane's offsets pos - key are consecutive for consecutive keys, so each
+          // lane collects its hits into (at most three) words first.
+          const unsigned same_head = __match_any_sync(0xffffffffu, hl);
+          const int leader = __ffs(same_head) - 1;
+          const int kbase = j0 + half * 64;
+          const int64_t vbit0 = static_cast<int64_t>(tok0) + kbase;   // bit of key kbase
+          const int64_t vw0 = vbit0 >> 5;
+          const int64_t sbit_hi = static_cast<int64_t>(tok0) + pos - kbase;  // offset of key kbase
+          const int64_t sw0 = (sbit_hi - 63) >> 5;
+          uint32_t v0 = 0, v1 = 0, v2 = 0, s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            if (j >= nv) continue;
             const float x = __uint_as_float(r[j]) * sl2;
-            const int key = j0 + half * 64 + j;
-            if (x >= bv) {
-              const int64_t bi = static_cast<int64_t>(tok0) + key;
-              atomicOr(vrow + (bi >> 5), 1u << (bi & 31));
+            const bool hv = j < nv && x >= bv;
+            const bool hs = j < nv && x >= bs;
+            if (__ballot_sync(0xffffffffu, hv) & same_head) {
+              const int64_t bit = vbit0 + j;
+              const int idx = static_cast<int>((bit >> 5) - vw0);
+              const uint32_t m = 1u << (bit & 31);
+              if (idx == 0) v0 |= m; else if (idx == 1) v1 |= m; else v2 |= m;
             }
-            if (x >= bs) {
-              const int64_t bi = static_cast<int64_t>(tok0) + pos - key;
-              atomicOr(srow + (bi >> 5), 1u << (bi & 31));
+            if (hs) {
+              const int64_t bit = sbit_hi - j;
+              const int idx = static_cast<int>((bit >> 5) - sw0);
+              const uint32_t m = 1u << (bit & 31);
+              if (idx == 0) s0 |= m; else if (idx == 1) s1 |= m; else s2 |= m;
             }
           }
+          if (lane == leader) {
+            if (v0) atomicOr(vrow + vw0, v0);
+            if (v1) atomicOr(vrow + vw0 + 1, v1);
+            if (v2) atomicOr(vrow + vw0 + 2, v2);
+          }
+          if (s0) atomicOr(srow + sw0, s0);
+          if (s1) atomicOr(srow + sw0 + 1, s1);
+          if (s2) atomicOr(srow + sw0 + 2, s2);
         }
       }
     }
