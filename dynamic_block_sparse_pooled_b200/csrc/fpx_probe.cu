@@ -61,11 +61,23 @@ constexpr uint32_t kQTileBytesBf16 = kRowsPerTile * kHeadDim * 2;  // 32 KB
 constexpr uint32_t kKSlotBytes = kKeys * kHeadDim * 2;             // 32 KB (bf16; e4m3 uses half)
 constexpr uint32_t kBoxBytes = 128 * 128;                          // 128 rows x 128 B
 
+// Per tile count: K ring slots and S buffers in TMEM (two S buffers, so that the next block's
+// MMA overlaps this block's row work, where two fit in the 512 TMEM columns).
+template <int kTiles>
+struct PLayout {
+  static constexpr int kBufs = kTiles <= 2 ? 2 : 1;
+  static constexpr int kSlots = kTiles <= 2 ? 3 : 2;
+  static constexpr uint32_t kTmemCols = kBufs * kTiles * 128 <= 128   ? 128
+                                        : kBufs * kTiles * 128 <= 256 ? 256
+                                                                      : 512;
+};
+
 __host__ __device__ constexpr size_t probe_smem_bytes(int tiles) {
-  return static_cast<size_t>(tiles) * kQTileBytesBf16 + 2 * kKSlotBytes + 256 + 1024;
+  return static_cast<size_t>(tiles) * kQTileBytesBf16 +
+         static_cast<size_t>(tiles <= 2 ? 3 : 2) * kKSlotBytes + 256 + 1024;
 }
 
-enum PBar { kPKFull = 0, kPKEmpty = 2, kPSFull = 4, kPSFree = 5, kPDrain = 6, kPNumBars = 7 };
+enum PBar { kPKFull = 0, kPKEmpty = 3, kPSFull = 6, kPSFree = 8, kPDrain = 10, kPNumBars = 11 };
 
 template <bool kFp8>
 struct PCfg {
@@ -164,16 +176,16 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
                   uint32_t* __restrict__ sbits, StatusBlock* st) {
   pdl_enter();  // after the previous kernel on the stream
   using C = PCfg<kFp8>;
+  using L = PLayout<kTiles>;
   constexpr int kRowThreads = kTiles * 128;
   constexpr int kCtrlWarp = kTiles * 4;
-  constexpr uint32_t kTmemCols = kTiles == 1 ? 128 : kTiles == 2 ? 256 : 512;
   if (!*tab.valid) return;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - raw_u32);
   const uint32_t off_k = kTiles * C::kTileBytes;
-  const uint32_t off_bar = off_k + 2 * kKSlotBytes;
+  const uint32_t off_bar = off_k + L::kSlots * kKSlotBytes;
   const uint32_t bar0 = sbase + off_bar;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + off_bar + 8 * kPNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + off_bar + 8 * kPNumBars + 4);
@@ -191,12 +203,14 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
   const int rows = p.group * a.n_probe;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < L::kSlots; ++i) {
       mbar_init(bar(kPKFull + i), 1);
       mbar_init(bar(kPKEmpty + i), 1);
     }
-    mbar_init(bar(kPSFull), 1);
-    mbar_init(bar(kPSFree), kRowThreads / 32);
+    for (int i = 0; i < L::kBufs; ++i) {
+      mbar_init(bar(kPSFull + i), 1);
+      mbar_init(bar(kPSFree + i), kRowThreads / 32);
+    }
     mbar_init(bar(kPDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -224,7 +238,7 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
   if (warp == kCtrlWarp) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -233,89 +247,104 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kCtrlWarp) {
-    // ---- TMA loads of the chunk's K blocks and the QK^T MMAs (one elected lane) ----------
+    // ---- TMA loads of the chunk's K blocks (a kSlots ring) and the QK^T MMAs into kBufs
+    //      S buffers (one elected lane) -------------------------------------------------------
     constexpr unsigned kFull = 0xffffffffu;
     const uint64_t qdesc0 = smem_desc_sw128(sbase, 16, 1024);
     const uint64_t kdesc0 = smem_desc_sw128(sbase + off_k, 16, 1024);
     const int nblk = J1 - J0;
     bool ok = true;
-    // the first two blocks' loads up front
-    for (int e = 0; e < min(2, nblk); ++e) {
+    int loaded = 0;
+    auto load_block = [&](int idx) {  // block J0 + idx into ring slot idx % kSlots
+      const int slot = idx % L::kSlots;
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar(kPKFull + e), C::kTileBytes);
+        mbar_arrive_expect_tx(bar(kPKFull + slot), C::kTileBytes);
 #pragma unroll
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(sbase + off_k + e * kKSlotBytes + bx * kBoxBytes, &tmK, bar(kPKFull + e),
-                      bx * 128 / C::kElem, g, tok0 + (J0 + e) * kKeys);
+          tma_load_3d(sbase + off_k + slot * kKSlotBytes + bx * kBoxBytes, &tmK,
+                      bar(kPKFull + slot), bx * 128 / C::kElem, g, tok0 + (J0 + idx) * kKeys);
       }
       __syncwarp();
-    }
-    int loaded = min(2, nblk);
+    };
+    for (; loaded < min(L::kSlots, nblk); ++loaded) load_block(loaded);
     for (int e = 0; e < nblk && ok; ++e) {
-      const int slot = e & 1;
-      const uint32_t ph = (e >> 1) & 1;
-      if (!__all_sync(kFull, mbar_wait(bar(kPKFull + slot), ph, abort_flag))) { ok = false; break; }
-      // S is a single TMEM buffer: the row threads must have read the previous block's S
-      if (e > 0 &&
-          !__all_sync(kFull, mbar_wait(bar(kPSFree), (e - 1) & 1, abort_flag))) { ok = false; break; }
+      const int slot = e % L::kSlots;
+      const int buf = e % L::kBufs;
+      if (!__all_sync(kFull, mbar_wait(bar(kPKFull + slot), (e / L::kSlots) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      // the row threads must have read block e - kBufs's S out of this buffer
+      if (e >= L::kBufs &&
+          !__all_sync(kFull, mbar_wait(bar(kPSFree + buf), ((e - L::kBufs) / L::kBufs) & 1,
+                                       abort_flag))) {
+        ok = false;
+        break;
+      }
       if (elect_one()) {
         tc_fence_after();
         const uint64_t kdesc = kdesc0 + ((slot * kKSlotBytes) >> 4);
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
           const uint64_t qdesc = qdesc0 + ((t * C::kTileBytes) >> 4);
+          const uint32_t dcol = tmem + (buf * kTiles + t) * 128;
 #pragma unroll
           for (int kk = 0; kk < C::kSteps; ++kk) {
             const uint64_t off = koff<kFp8>(kk) >> 4;
-            if (kFp8) mma_f8_ss(tmem + t * 128, qdesc + off, kdesc + off, C::kIdesc, kk > 0);
-            else mma_f16_ss(tmem + t * 128, qdesc + off, kdesc + off, C::kIdesc, kk > 0);
+            if (kFp8) mma_f8_ss(dcol, qdesc + off, kdesc + off, C::kIdesc, kk > 0);
+            else mma_f16_ss(dcol, qdesc + off, kdesc + off, C::kIdesc, kk > 0);
           }
         }
-        mma_commit(bar(kPSFull));
+        mma_commit(bar(kPSFull + buf));
         mma_commit(bar(kPKEmpty + slot));
       }
       __syncwarp();
-      // refill this slot with block e + 2 once the MMAs above have read it
-      if (loaded < nblk) {
-        if (!__all_sync(kFull, mbar_wait(bar(kPKEmpty + slot), ph, abort_flag))) { ok = false; break; }
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(kPKFull + slot), C::kTileBytes);
-#pragma unroll
-          for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(sbase + off_k + slot * kKSlotBytes + bx * kBoxBytes, &tmK,
-                        bar(kPKFull + slot), bx * 128 / C::kElem, g, tok0 + loaded * kKeys + J0 * kKeys);
+      // refill: block `loaded` (= e + kSlots - 1 in steady state) takes the slot of block
+      // loaded - kSlots <= e - 1, whose MMA went out an iteration ago, after block e's MMA is
+      // already queued behind it
+      if (loaded < nblk && loaded <= e + L::kSlots - 1) {
+        const int prev = loaded - L::kSlots;
+        if (!__all_sync(kFull, mbar_wait(bar(kPKEmpty + prev % L::kSlots),
+                                         (prev / L::kSlots) & 1, abort_flag))) {
+          ok = false;
+          break;
         }
-        __syncwarp();
+        load_block(loaded);
         ++loaded;
       }
     }
     if (!ok) *abort_flag = 1;
     // drain: the loads this warp issued, then every MMA, before TMEM is released
     volatile int never = 0;
-    for (int e = max(0, loaded - 2); e < loaded; ++e)
-      mbar_wait(bar(kPKFull + (e & 1)), (e >> 1) & 1, &never);
+    for (int e = max(0, loaded - L::kSlots); e < loaded; ++e)
+      mbar_wait(bar(kPKFull + e % L::kSlots), (e / L::kSlots) & 1, &never);
     if (elect_one()) mma_commit(bar(kPDrain));
     mbar_wait(bar(kPDrain), 0, &never);
   } else if (tid < kRowThreads) {
     // ---- one probe row per thread ---------------------------------------------------------
     const int tile = row >> 7;
-    const uint32_t taddr = tmem + tile * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int h = g * p.group + hl;
     float sl2 = p.scale * 1.4426950408889634f;
     if (kFp8 && row_valid) sl2 *= p.q_scale[h] * p.k_scale[g];
     float mrun = -CUDART_INF_F, lrun = 0.f;
+    // marks: bounds in raw score units (s * sl2 >= b  <=>  s >= b / sl2, sl2 > 0)
     float bv = CUDART_INF_F, bs = CUDART_INF_F;
     if (kMark && row_valid) {
       const float2 b = bound[(static_cast<int64_t>(s) * p.hq + h) * a.n_probe + pp];
-      bv = a.all_v ? CUDART_INF_F : b.x;  // alpha == 0 is filled elsewhere
-      bs = a.all_s ? CUDART_INF_F : b.y;
+      bv = a.all_v ? CUDART_INF_F : b.x / sl2;  // alpha == 0 is filled elsewhere
+      bs = a.all_s ? CUDART_INF_F : b.y / sl2;
     }
     uint32_t* vrow = vbits + static_cast<int64_t>(h) * a.words;
     uint32_t* srow = sbits + static_cast<int64_t>(h) * a.words;
+    const unsigned same_head = kMark ? __match_any_sync(0xffffffffu, hl) : 0u;
+    const int leader = __ffs(same_head) - 1;
     bool ok = true;
     for (int e = 0; e < J1 - J0; ++e) {
-      if (!mbar_wait(bar(kPSFull), e & 1, abort_flag)) { ok = false; break; }
+      const int buf = e % L::kBufs;
+      if (!mbar_wait(bar(kPSFull + buf), (e / L::kBufs) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t taddr = tmem + (buf * kTiles + tile) * 128 + lane_base;
       const int j0 = (J0 + e) * kKeys;
       const int nvis = row_valid ? min(kKeys, pos - j0 + 1) : 0;  // keys j0 .. pos of this block
       // the S row in two halves of 64 columns (register budget of up to 4 tiles x 128 threads)
@@ -329,7 +358,7 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
         if (half == 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPSFree));  // S may be overwritten by the next block
+          if (lane == 0) mbar_arrive(bar(kPSFree + buf));  // the buffer may be overwritten
         }
         const int nv = min(64, nvis - half * 64);  // visible columns of this half
         if (!kMark) {
@@ -346,46 +375,50 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
           lrun = lrun * ex2_approx(mrun - mnew) + sum;  // mrun = -inf: 0 * 0
           mrun = mnew;
         } else {
-          // Marks, gathered before the atomics.  Verticals: the key column is the same for
-          // every lane, so a vote per column among the lanes of one Q head (a warp holds the
-          // probe rows of several heads when n_probe is not a multiple of 32) collects that
-          // head's hits, and its first lane sets them with one atomicOr per 32-bit word.
-          // Slashes: a lane's offsets pos - key are consecutive for consecutive keys, so each
-          // lane collects its hits into (at most three) words first.
-          const unsigned same_head = __match_any_sync(0xffffffffu, hl);
-          const int leader = __ffs(same_head) - 1;
-          const int kbase = j0 + half * 64;
-          const int64_t vbit0 = static_cast<int64_t>(tok0) + kbase;   // bit of key kbase
-          const int64_t vw0 = vbit0 >> 5;
-          const int64_t sbit_hi = static_cast<int64_t>(tok0) + pos - kbase;  // offset of key kbase
-          const int64_t sw0 = (sbit_hi - 63) >> 5;
-          uint32_t v0 = 0, v1 = 0, v2 = 0, s0 = 0, s1 = 0, s2 = 0;
+          // Branch-free marks: bit j of (vlo, vhi) / (slo, shi) = column j of this half is
+          // above the vertical / slash bound.  Verticals: the key column is the same for every
+          // lane, so the head's lanes OR their masks together (a warp holds the probe rows of
+          // several heads when n_probe is not a multiple of 32) and the head's first lane sets
+          // the bits with one atomicOr per 32-bit word.  Slashes: a lane's columns j map to the
+          // consecutive offsets pos - key, so its mask, bit-reversed, is a bit range of the
+          // slash row; it is OR-ed in word by word (hits are rare).
+          uint32_t vlo = 0, vhi = 0, slo = 0, shi = 0;
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            const float x = __uint_as_float(r[j]) * sl2;
-            const bool hv = j < nv && x >= bv;
-            const bool hs = j < nv && x >= bs;
-            if (__ballot_sync(0xffffffffu, hv) & same_head) {
-              const int64_t bit = vbit0 + j;
-              const int idx = static_cast<int>((bit >> 5) - vw0);
-              const uint32_t m = 1u << (bit & 31);
-              if (idx == 0) v0 |= m; else if (idx == 1) v1 |= m; else v2 |= m;
-            }
-            if (hs) {
-              const int64_t bit = sbit_hi - j;
-              const int idx = static_cast<int>((bit >> 5) - sw0);
-              const uint32_t m = 1u << (bit & 31);
-              if (idx == 0) s0 |= m; else if (idx == 1) s1 |= m; else s2 |= m;
-            }
+            const float x = __uint_as_float(r[j]);
+            const uint32_t vis = j < nv ? 1u : 0u;
+            const uint32_t hv = (x >= bv ? 1u : 0u) & vis, hs = (x >= bs ? 1u : 0u) & vis;
+            if (j < 32) { vlo |= hv << j; slo |= hs << j; }
+            else { vhi |= hv << (j - 32); shi |= hs << (j - 32); }
           }
-          if (lane == leader) {
-            if (v0) atomicOr(vrow + vw0, v0);
-            if (v1) atomicOr(vrow + vw0 + 1, v1);
-            if (v2) atomicOr(vrow + vw0 + 2, v2);
+          vlo = __reduce_or_sync(0xffffffffu & same_head, vlo);
+          vhi = __reduce_or_sync(0xffffffffu & same_head, vhi);
+          const int kbase = j0 + half * 64;
+          if (lane == leader && (vlo | vhi)) {
+            // keys kbase .. kbase + 63 at bits vbit0 .. vbit0 + 63 of the head's row
+            const int64_t vbit0 = static_cast<int64_t>(tok0) + kbase;
+            const int64_t w0 = vbit0 >> 5;
+            const int sh = static_cast<int>(vbit0 & 31);
+            const uint32_t x0 = vlo << sh;
+            const uint32_t x1 = sh ? (vhi << sh) | (vlo >> (32 - sh)) : vhi;
+            const uint32_t x2 = sh ? vhi >> (32 - sh) : 0u;
+            if (x0) atomicOr(vrow + w0, x0);
+            if (x1) atomicOr(vrow + w0 + 1, x1);
+            if (x2) atomicOr(vrow + w0 + 2, x2);
           }
-          if (s0) atomicOr(srow + sw0, s0);
-          if (s1) atomicOr(srow + sw0 + 1, s1);
-          if (s2) atomicOr(srow + sw0 + 2, s2);
+          if (slo | shi) {
+            // column j <-> offset pos - kbase - j: reversed, bit k <-> offset pos - kbase - 63 + k
+            const uint32_t rlo = __brev(shi), rhi = __brev(slo);
+            const int64_t sbit0 = static_cast<int64_t>(tok0) + pos - kbase - 63;
+            const int64_t w0 = sbit0 >> 5;  // floor (bits below the row's start are zero)
+            const int sh = static_cast<int>(sbit0 & 31);
+            const uint32_t x0 = rlo << sh;
+            const uint32_t x1 = sh ? (rhi << sh) | (rlo >> (32 - sh)) : rhi;
+            const uint32_t x2 = sh ? rhi >> (32 - sh) : 0u;
+            if (x0) atomicOr(srow + w0, x0);
+            if (x1) atomicOr(srow + w0 + 1, x1);
+            if (x2) atomicOr(srow + w0 + 2, x2);
+          }
         }
       }
     }
@@ -401,7 +434,7 @@ probe_pass_kernel(const __grid_constant__ CUtensorMap tmK, ProblemDesc p, ProbeA
   __syncthreads();
   if (warp == kCtrlWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
