@@ -36,7 +36,9 @@
 //
 // Softmax: exp2 domain, lazy rescale (the reference max only moves when the block max exceeds it
 // by more than 2^8), the S row read from TMEM in two halves (the second in flight while the first
-// is reduced) and P written back in two halves (the first while the second is computed).  Every
+// is reduced) and P written back in two halves (the first while the second is computed); e4m3
+// forms P in the same pass as the block max once a reference exists, and redoes the block in two
+// passes only when the max moves the reference.  Every
 // wait is bounded: a broken pipeline records FPX_ERR_TIMEOUT, drains its own TMA loads and MMAs,
 // releases TMEM and exits.
 #include <cuda.h>
@@ -629,71 +631,105 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         s_phase ^= 1;
         tc_fence_after();
         const bool diag = (J == w.I);
+        // token causal mask (key column > query row) and token mask of one 64-column half
+        auto mask_half = [&](uint32_t* x, int j0) {
+          if (diag) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              if (j0 + j > row) x[j] = __float_as_uint(-CUDART_INF_F);
+          }
+          if (kMask) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              if (!((am[(j0 + j) >> 5] >> ((j0 + j) & 31)) & 1u)) x[j] = __float_as_uint(-CUDART_INF_F);
+          }
+        };
         // the whole S row of this thread: 128 fp32 in registers (one TMEM read)
         uint32_t r[128];
-        tmem_ld32(tS, r);
-        tmem_ld32(tS + 32, r + 32);
-        tmem_wait_ld(r);
-        tmem_wait_ld(r + 32);
-        // second half in flight while the first half is masked and reduced
-        tmem_ld32(tS + 64, r + 64);
-        tmem_ld32(tS + 96, r + 96);
-        if (diag) {  // token causal mask: key column > query row
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
-        }
-        if (kMask) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (!((am[j >> 5] >> (j & 31)) & 1u)) r[j] = __float_as_uint(-CUDART_INF_F);
-        }
-        const float mx_lo = row_max64(r);
-        tmem_wait_ld(r + 64);
-        tmem_wait_ld(r + 96);
-        if (diag) {
-#pragma unroll
-          for (int j = 64; j < 128; ++j)
-            if (j > row) r[j] = __float_as_uint(-CUDART_INF_F);
-        }
-        if (kMask) {
-#pragma unroll
-          for (int j = 64; j < 128; ++j)
-            if (!((am[j >> 5] >> (j & 31)) & 1u)) r[j] = __float_as_uint(-CUDART_INF_F);
-        }
-        // finite unless kMask: key 0 of a block row is always visible without the token mask;
-        // with it a row may see no key yet (m_ref = -inf), and -inf then stands for "none"
-        const float mx = fmaxf(mx_lo, row_max64(r + 64)) * sl2;
-        // lazy rescale: move the reference max only when the block max exceeds it by > 2^8
-        float corr = 1.f;
-        if (mx > m_ref + kRescaleLog2) {
-          corr = ex2_approx(m_ref - mx);  // 0 for the first block
-          l_run *= corr;
-          m_ref = mx;
-        }
-        if (it > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
-          // O_t is stable: the previous P*V into it completed before S_t was written
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tO + c * 32, ov);
-            tmem_wait_ld(ov);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * corr);
-            tmem_st32(tO + c * 32, ov);
+        float rs = 0.f;
+        // e4m3: once the reference max is set (every lane of the warp), P is formed against it
+        // in the same pass that takes the block max; the lazy-rescale rule keeps that P whenever
+        // the block max stays within 2^8 of the reference, which is the rule's own no-rescale
+        // case, so the result is the one the two-pass order gives.  Otherwise nothing has been
+        // stored yet, S is still in TMEM, and the warp redoes the block in two passes.  (bf16
+        // keeps the two-pass order: its P is twice as many TMEM columns, and storing the first
+        // half while the second is formed was measured to be worth more than the single pass.)
+        const bool spec = kFp8 && it > 0 && __all_sync(kFull, m_ref != -CUDART_INF_F);
+        bool redo = !spec;
+        if (spec) {
+          tmem_ld32(tS, r);
+          tmem_ld32(tS + 32, r + 32);
+          tmem_wait_ld(r);
+          tmem_wait_ld(r + 32);
+          tmem_ld32(tS + 64, r + 64);
+          tmem_ld32(tS + 96, r + 96);
+          mask_half(r, 0);
+          const float mx_lo = row_max64(r);
+          rs = softmax_part_to_p<kFp8, 0, 64>(r, sl2, -m_ref);
+          tmem_wait_ld(r + 64);
+          tmem_wait_ld(r + 96);
+          mask_half(r + 64, 64);
+          const float mx = fmaxf(mx_lo, row_max64(r + 64)) * sl2;
+          rs += softmax_part_to_p<kFp8, 64, 64>(r, sl2, -m_ref);
+          redo = __any_sync(kFull, mx > m_ref + kRescaleLog2);
+          if (!redo) {
+            if (kFp8) {
+              tmem_st16(tS, r);
+              tmem_st16(tS + 16, r + 16);
+            } else {
+              tmem_st32(tS, r);
+              tmem_st32(tS + 32, r + 32);
+            }
           }
         }
-        // P = exp2(s * sl2 - m_ref), packed in place and written over S
-        // first half of P stored while the second half is computed
-        // (a row that no key has reached yet: exponents of -inf, P = 0, and the weights the
-        // FMA-pipe exp2 gives them are cleared by the rescale that its first key triggers)
-        const float neg_m = (kMask && m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
-        float rs = softmax_part_to_p<kFp8, 0, 64>(r, sl2, neg_m);
-        if (kFp8) tmem_st16(tS, r);
-        else tmem_st32(tS, r);
-        rs += softmax_part_to_p<kFp8, 64, 64>(r, sl2, neg_m);
-        if (kFp8) tmem_st16(tS + 16, r + 16);
-        else tmem_st32(tS + 32, r + 32);
+        if (redo) {
+          tmem_ld32(tS, r);
+          tmem_ld32(tS + 32, r + 32);
+          tmem_wait_ld(r);
+          tmem_wait_ld(r + 32);
+          // second half in flight while the first half is masked and reduced
+          tmem_ld32(tS + 64, r + 64);
+          tmem_ld32(tS + 96, r + 96);
+          mask_half(r, 0);
+          const float mx_lo = row_max64(r);
+          tmem_wait_ld(r + 64);
+          tmem_wait_ld(r + 96);
+          mask_half(r + 64, 64);
+          // finite unless kMask: key 0 of a block row is always visible without the token
+          // mask; with it a row may see no key yet (m_ref = -inf), and -inf then stands for
+          // "none"
+          const float mx = fmaxf(mx_lo, row_max64(r + 64)) * sl2;
+          // lazy rescale: move the reference max only when the block max exceeds it by > 2^8
+          float corr = 1.f;
+          if (mx > m_ref + kRescaleLog2) {
+            corr = ex2_approx(m_ref - mx);  // 0 for the first block
+            l_run *= corr;
+            m_ref = mx;
+          }
+          if (it > 0 && __any_sync(kFull, corr != 1.f)) {
+            // O_t is stable: the previous P*V into it completed before S_t was written
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t ov[32];
+              tmem_ld32(tO + c * 32, ov);
+              tmem_wait_ld(ov);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * corr);
+              tmem_st32(tO + c * 32, ov);
+            }
+          }
+          // P = exp2(s * sl2 - m_ref), packed in place and written over S
+          // first half of P stored while the second half is computed
+          // (a row that no key has reached yet: exponents of -inf, P = 0, and the weights the
+          // FMA-pipe exp2 gives them are cleared by the rescale that its first key triggers)
+          const float neg_m = (kMask && m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+          rs = softmax_part_to_p<kFp8, 0, 64>(r, sl2, neg_m);
+          if (kFp8) tmem_st16(tS, r);
+          else tmem_st32(tS, r);
+          rs += softmax_part_to_p<kFp8, 64, 64>(r, sl2, neg_m);
+          if (kFp8) tmem_st16(tS + 16, r + 16);
+          else tmem_st32(tS + 32, r + 32);
+        }
         l_run += rs;
         tmem_wait_st();
         tc_fence_before();

@@ -28,8 +28,9 @@ CASES = {
 }
 
 
-def run_case(w, alpha, sink=1, window=1):
-    data = generate(w, workers=4)
+def run_case(w, alpha, sink=1, window=1, data=None):
+    if data is None:
+        data = generate(w, workers=4)
     q64, k64, v64 = PT.oracle_inputs(data)
     cu = data["cu_seqlens"]
     dev = PT.to_device(data)
@@ -173,3 +174,39 @@ def test_empty_problem():
     k = torch.zeros((0, 2, 128), dtype=torch.bfloat16, device="cuda")
     out = fpx.prefill(q, k, k, 128, 0.1)
     assert out["o"].shape == (0, 4, 128) and int(out["nnz"].item()) == 0
+
+
+def rising_maxima_data(dtype):
+    """Logits that rise by ~12 log2 units per key block for about half of the query rows (the
+    sign of a fixed query component drawn per row and head, so mixed inside every warp of 32
+    rows) and fall for the rest: a rising row's block maximum passes the lazy-rescale threshold
+    (2^8) at every block after its first, a falling row's never does."""
+    w = BASE.with_(seqlens=(1000, 700), hq=4, hkv=2)
+    data = generate(w, workers=4)
+    cu = data["cu_seqlens"]
+    q, k, v = data["q"].float(), data["k"].float(), data["v"].float()
+    g = torch.Generator().manual_seed(1234)
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        blk = (torch.arange(b - a, dtype=torch.float32) // w.block).view(-1, 1)
+        k[a:b, :, 0] = 8.0 * blk
+        sign = torch.where(torch.rand(b - a, w.hq, generator=g) < 0.5, -1.0, 1.0)
+        q[a:b, :, 0] = 12.0 * sign
+    if dtype == "bf16":
+        data.update(q=q.to(torch.bfloat16), k=k.to(torch.bfloat16), v=v.to(torch.bfloat16))
+    else:
+        from gen.synthetic import _quant_e4m3
+        w = w.with_(dtype="e4m3")
+        (q8, qs), (k8, ks), (v8, vs) = _quant_e4m3(q), _quant_e4m3(k), _quant_e4m3(v)
+        data.update(q=q8, k=k8, v=v8, q_scale=qs, k_scale=ks, v_scale=vs)
+    data["workload"] = w
+    return w, data
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("alpha", [0.0, 0.3])
+def test_rising_maxima_rescale_mid_row(dtype, alpha):
+    w, data = rising_maxima_data(dtype)
+    res = run_case(w, alpha, data=data)
+    assert res["path"] == 1
+    print(dtype, alpha, res)
