@@ -45,9 +45,9 @@ KERNELS_PER_STEP = 10  # plan+pool+score, plan+count+scan+emit, plan+order+atten
 ATTN_SOURCES = ("dynamic_block_sparse_pooled_b200/csrc/fpx_attn_sm100.cu",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_sm100.cuh",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_common.cuh")
-ATTN_TRAFFIC_DIGEST = "6b793b6fb7ca1753bdc8ad6f8cb0608a19ff208e02c1a225b10169018174f519"
+ATTN_TRAFFIC_DIGEST = "23f8956b12ed3efcff1f745b00ee6c06cefc38e88af5ccb44e97a6e6eab99120"
 ATTN_TRAFFIC = {
-    "llama8b_bf16_n131072": 3303332864 + 1180280320,
+    "llama8b_bf16_n131072": 3299871744 + 1179726848,
 }
 
 
