@@ -111,6 +111,67 @@ def pairs(w) -> int:
     return sum((-(-n // w.block)) * (-(-n // w.block) + 1) // 2 for n in w.seqlens)
 
 
+NEAR_REL = 1e-3  # near-threshold band: |exp(s - m) - alpha| <= NEAR_REL * alpha
+
+
+def selection_stats(scores, row_ptr, col_idx, cu, hq: int, hkv: int, block: int, alpha: float,
+                    sink: int, window: int) -> dict:
+    """Figures of one selection, from the device tensors after the timed region:
+
+    * near_threshold_blocks: causal blocks not forced by sink / window whose ratio exp(s - m_I)
+      (m_I = the row maximum of the pooled scores) lies within NEAR_REL * alpha of alpha — the
+      blocks where an fp32 and an fp64 decision may both be right;
+    * kv_tile_loads: K / V tile pairs the attention loads, one per block in the union of the
+      two Q heads of a work unit (heads 2p and 2p + 1 of a KV group; an odd last head alone);
+    * union_excess_tiles: tiles multiplied for a head that did not keep them (0: the kernel
+      issues a tile's MMAs only for the heads that kept it; the union only shares the loads).
+    scores: fp32 [hq * TRI] triangular-packed; row_ptr / col_idx: the CSR of fpx_select."""
+    dev = scores.device
+    nbs = [-(-(int(cu[i + 1]) - int(cu[i])) // block) for i in range(len(cu) - 1)]
+    row_i, row_start, tri = [], [], 0
+    for nb in nbs:
+        for i in range(nb):
+            row_i.append(i)
+            row_start.append(tri + i * (i + 1) // 2)
+        tri += nb * (nb + 1) // 2
+    rows_h = len(row_i)
+    out = {"near_threshold_blocks": 0, "kv_tile_loads": 0, "union_excess_tiles": 0}
+    if rows_h == 0 or tri == 0:
+        return out
+    row_i = torch.tensor(row_i, dtype=torch.int64, device=dev)
+    row_start = torch.tensor(row_start, dtype=torch.int64, device=dev)
+    # row (within a head) of every triangular element, and its block indices I, J
+    elem_row = torch.repeat_interleave(torch.arange(rows_h, device=dev), row_i + 1)
+    elem_j = torch.arange(tri, device=dev) - row_start[elem_row]
+    elem_i = row_i[elem_row]
+    s = scores[:hq * tri].view(hq, tri).double()
+    if alpha > 0:
+        m = torch.full((hq, rows_h), float("-inf"), dtype=torch.float64, device=dev)
+        m = m.scatter_reduce(1, elem_row.expand(hq, -1), s, reduce="amax", include_self=True)
+        ratio = torch.exp(s - m.gather(1, elem_row.expand(hq, -1)))
+        forced = (elem_j < sink) | (elem_j > elem_i - window)
+        near = (~forced) & ((ratio - alpha).abs() <= NEAR_REL * alpha)
+        out["near_threshold_blocks"] = int(near.sum().item())
+    # kept flags in the triangular layout, from the CSR
+    rp = row_ptr.to(torch.int64)
+    nnz = int(rp[-1].item())
+    kept = torch.zeros(hq * tri, dtype=torch.bool, device=dev)
+    if nnz > 0:
+        counts = rp[1:] - rp[:-1]
+        row_of = torch.repeat_interleave(torch.arange(hq * rows_h, device=dev), counts)
+        pos = (row_of // rows_h) * tri + row_start[row_of % rows_h] + col_idx[:nnz].to(torch.int64)
+        kept[pos] = True
+    kept = kept.view(hq, tri)
+    g = hq // hkv
+    loads = 0
+    for kvh in range(hkv):
+        for h0 in range(kvh * g, (kvh + 1) * g, 2):
+            u = kept[h0] | kept[h0 + 1] if h0 + 1 < (kvh + 1) * g else kept[h0]
+            loads += int(u.sum().item())
+    out["kv_tile_loads"] = loads
+    return out
+
+
 class ClockSampler:
     """Samples the SM clock and the clock-event (throttle) reasons during the timed region, with
     NVML every 10 ms (short regions get at least one sample, taken at exit)."""
@@ -361,7 +422,16 @@ class Prefill:
         res = self.metrics([a.elapsed_time(b) for a, b, c in timing],
                            [b.elapsed_time(c) for a, b, c in timing], n_kept)
         res["clocks"] = clk.summary()
+        res.update(self.selection())
         return res
+
+    def selection(self):
+        w = self.w
+        st = selection_stats(self.scores, self.row_ptr, self.col_idx, self.cu, w.hq, w.hkv,
+                             w.block, w.alpha, w.sink_blocks, w.window_blocks)
+        n_kept = int(self.nnz.item())
+        st["kv_loads_per_kept_tile"] = round(st["kv_tile_loads"] / n_kept, 4) if n_kept else None
+        return st
 
 
 def sub_records(fpx, args, device, sdpa_ms_128k):
@@ -558,7 +628,7 @@ def run_ours(args, rank, world, device):
         "config": config_of(w, world),
         "attn_ms": m["attn_ms"], "search_ms": m["search_ms"],
         "attn_dense_equiv_tflops": m["attn_dense_equiv_tflops"],
-        "density": m["density"], "nnz": n_kept,
+        "density": m["density"], "nnz": n_kept, "selection": run.selection(),
         "search_bytes": m["search_bytes"], "search_scores_readback_bytes": 4 * w.hq * pairs(w),
         "search_gbs": m["search_gbs"], "search_hbm_frac": m["search_hbm_frac"],
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": achieved,

@@ -59,8 +59,14 @@ constexpr int kTileM = 128;   // query rows per tile (= block)
 constexpr int kTileN = 128;   // keys per block
 constexpr int kHeadDim = 128;
 constexpr int kThreads = 384;
-constexpr int kSoftmaxRegs = 208;  // 256 x 208 + 128 x 80 <= 384 x 168 (registers at launch)
-constexpr int kOtherRegs = 80;
+// softmax / other warpgroups' registers after setmaxnreg: 256 x S + 128 x O <= 384 x 168 (the
+// registers at launch), both multiples of 8
+#ifndef FPX_SOFTMAX_REGS
+#define FPX_SOFTMAX_REGS 208
+#endif
+constexpr int kSoftmaxRegs = FPX_SOFTMAX_REGS;
+constexpr int kOtherRegs = (384 * 168 - 256 * kSoftmaxRegs) / 128 / 8 * 8;
+static_assert(kOtherRegs >= 24 && kSoftmaxRegs % 8 == 0 && kSoftmaxRegs <= 256, "register split");
 constexpr int kMmaWarp = 8;    // issues every MMA; allocates TMEM
 constexpr int kLoadWarp = 10;
 constexpr uint32_t kSlotBytes = 32768;  // one 128 x 128 bf16 tile

@@ -85,3 +85,44 @@ def test_traffic_is_reported_only_for_the_measured_sources(monkeypatch):
     # kernel sources that differ from the captured ones: null
     monkeypatch.setattr(bench, "ATTN_TRAFFIC_DIGEST", "0" * 64)
     assert bench.attn_traffic("llama8b_bf16_n131072") is None
+
+
+@pytest.mark.parametrize("alpha,sink,window", [(1.0, 1, 1), (1.0, 0, 2), (0.0, 1, 1)])
+def test_selection_stats_match_the_oracle(alpha, sink, window):
+    """bench.selection_stats on a varlen problem (a ragged tail and a zero-length sequence, odd
+    GQA group): the near-threshold count equals the oracle's near mask, and the K/V tile loads
+    equal the brute-force union of each unit's two heads' kept blocks."""
+    import numpy as np
+    from oracle import fpx_oracle as O
+    rng = np.random.default_rng(7)
+    seqlens, hq, hkv, d, block = (70, 0, 33, 128), 6, 2, 16, 16
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    t = int(cu[-1])
+    q = rng.standard_normal((t, hq, d)) * 3.0
+    k = rng.standard_normal((t, hkv, d))
+    sc = O.block_scores(q, k, cu, block)
+    if alpha > 0:
+        # put alpha beside the ratio of an unforced causal block so that the band is not empty
+        s0 = sc[0][1]  # sequence 0, Q head 1: [nb, nb]
+        I = s0.shape[0] - 1
+        J = I - window if sink <= I - window else 0
+        alpha = float(np.exp(s0[I, J] - s0[I, :I + 1].max())) * (1 + 4e-4)
+    keeps, nears = O.select(sc, alpha, sink, window)
+    if alpha > 0:
+        assert sum(int(n.sum()) for n in nears) >= 1
+    rp, ci = O.to_csr(keeps)
+    scores = torch.from_numpy(O.triangular_pack(sc).astype(np.float32).reshape(-1))
+    st = bench.selection_stats(scores, torch.from_numpy(rp.astype(np.int32)),
+                               torch.from_numpy(ci.astype(np.int32) if ci.size else
+                                                np.zeros(1, np.int32)),
+                               cu, hq, hkv, block, alpha, sink, window)
+    assert st["near_threshold_blocks"] == sum(int(n.sum()) for n in nears)
+    g = hq // hkv
+    loads = 0
+    for kp in keeps:  # [hq, nb, nb] per sequence
+        for kvh in range(hkv):
+            for h0 in range(kvh * g, (kvh + 1) * g, 2):
+                u = kp[h0] | kp[h0 + 1] if h0 + 1 < (kvh + 1) * g else kp[h0]
+                loads += int(u.sum())
+    assert st["kv_tile_loads"] == loads
+    assert st["union_excess_tiles"] == 0
