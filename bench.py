@@ -45,9 +45,9 @@ KERNELS_PER_STEP = 10  # plan+pool+score, plan+count+scan+emit, plan+order+atten
 ATTN_SOURCES = ("dynamic_block_sparse_pooled_b200/csrc/fpx_attn_sm100.cu",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_sm100.cuh",
                 "dynamic_block_sparse_pooled_b200/csrc/fpx_common.cuh")
-ATTN_TRAFFIC_DIGEST = "23f8956b12ed3efcff1f745b00ee6c06cefc38e88af5ccb44e97a6e6eab99120"
+ATTN_TRAFFIC_DIGEST = "f88c351c7ee3c84bab085496a3a55124c32d919be05b2a163c66a83baa3ea018"
 ATTN_TRAFFIC = {
-    "llama8b_bf16_n131072": 3299871744 + 1179726848,
+    "llama8b_bf16_n131072": 3301625856 + 1180681216,
 }
 
 
