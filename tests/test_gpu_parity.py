@@ -176,11 +176,14 @@ def test_empty_problem():
     assert out["o"].shape == (0, 4, 128) and int(out["nnz"].item()) == 0
 
 
-def rising_maxima_data(dtype):
+def rising_maxima_data(dtype, pattern="block"):
     """Logits that rise by ~12 log2 units per key block for about half of the query rows (the
     sign of a fixed query component drawn per row and head, so mixed inside every warp of 32
     rows) and fall for the rest: a rising row's block maximum passes the lazy-rescale threshold
-    (2^8) at every block after its first, a falling row's never does."""
+    (2^8) at every block after its first, a falling row's never does.  pattern "block" raises
+    whole blocks (the first 64 keys of a block already pass the threshold); "second_half"
+    raises only keys 64-127 of every block (the first 64 stay at the bottom), so the maximum
+    moves the reference in the second half of every block after the first."""
     w = BASE.with_(seqlens=(1000, 700), hq=4, hkv=2)
     data = generate(w, workers=4)
     cu = data["cu_seqlens"]
@@ -188,8 +191,13 @@ def rising_maxima_data(dtype):
     g = torch.Generator().manual_seed(1234)
     for s in range(len(cu) - 1):
         a, b = int(cu[s]), int(cu[s + 1])
-        blk = (torch.arange(b - a, dtype=torch.float32) // w.block).view(-1, 1)
-        k[a:b, :, 0] = 8.0 * blk
+        pos = torch.arange(b - a, dtype=torch.float32)
+        blk = (pos // w.block).view(-1, 1)
+        if pattern == "block":
+            k[a:b, :, 0] = 8.0 * blk
+        else:
+            upper = ((pos % w.block) >= w.block // 2).float().view(-1, 1)
+            k[a:b, :, 0] = 8.0 * (blk + 1.0) * upper
         sign = torch.where(torch.rand(b - a, w.hq, generator=g) < 0.5, -1.0, 1.0)
         q[a:b, :, 0] = 12.0 * sign
     if dtype == "bf16":
@@ -203,10 +211,11 @@ def rising_maxima_data(dtype):
     return w, data
 
 
+@pytest.mark.parametrize("pattern", ["block", "second_half"])
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
 @pytest.mark.parametrize("alpha", [0.0, 0.3])
-def test_rising_maxima_rescale_mid_row(dtype, alpha):
-    w, data = rising_maxima_data(dtype)
+def test_rising_maxima_rescale_mid_row(dtype, alpha, pattern):
+    w, data = rising_maxima_data(dtype, pattern)
     res = run_case(w, alpha, data=data)
     assert res["path"] == 1
     print(dtype, alpha, res)
