@@ -586,7 +586,7 @@ def run_ours(args, rank, world, device):
     host_lse = [torch.empty(run.lse.shape, dtype=run.lse.dtype, pin_memory=True)
                 for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    e2e_steps = max(3, min(args.steps, 6))
+    e2e_steps = max(3, args.steps)  # as many steps as the device-timed region
     for r in slots:  # warm both buffer sets
         r.step()
     torch.cuda.synchronize(device)
