@@ -42,6 +42,9 @@ MUTATIONS = {
         "near_band_absolute": ("np.abs(x - thr) <= O.NEAR_REL * thr", "np.abs(x - thr) <= O.NEAR_REL"),
         "token_rows_offset_sign": ("keys = j[isv[j] | iss[i - j]]", "keys = j[isv[j] | iss[j]]"),
         "token_rows_not_causal": ("j = np.arange(i + 1)", "j = np.arange(min(i + 2, n))"),
+        "probe_kv_head_modulo": ("k[start:start + n, h // g]", "k[start:start + n, h % k.shape[1]]"),
+        "probe_scale_dropped": ("logits = scale * (kk[:i + 1] @", "logits = (kk[:i + 1] @"),
+        "probe_rows_not_normalised": ("a[h, p, :i + 1] = e / e.sum()", "a[h, p, :i + 1] = e"),
     }),
 }
 

@@ -122,7 +122,24 @@ def check_token_rows_equal_full_token_mask_attention(PO=PO):
     assert np.isneginf(lse_r[1]) and not o_r[1].any()  # head 1, token 0: no key at all
 
 
-ALL_CHECKS = [check_near_threshold_band, check_token_rows_equal_full_token_mask_attention,
+def check_probe_rows_are_causal_softmax_rows(PO=PO):
+    # the probe rows are exact causal attention rows (FlashPrefill §3, query probes): against
+    # torch's softmax of the masked logits, with GQA (Q head h reads KV head h / (Hq / Hkv)) and
+    # a sequence that starts inside the token array
+    rng = np.random.default_rng(5)
+    t, hq, hkv, d, start, n, sc = 30, 4, 2, 8, 3, 25, 0.37
+    q, k = rng.standard_normal((t, hq, d)), rng.standard_normal((t, hkv, d))
+    pos = PO.probe_positions(n, 5)
+    a = PO.probe_attention(q, k, start, n, pos, sc, hq // hkv)
+    causal = torch.ones(n, n, dtype=torch.bool).tril()
+    for h in range(hq):
+        qq = torch.from_numpy(q[start:start + n, h])
+        kk = torch.from_numpy(k[start:start + n, h * hkv // hq])
+        ref = torch.softmax((sc * qq @ kk.T).masked_fill(~causal, float("-inf")), dim=-1)
+        assert np.allclose(a[h], ref[torch.from_numpy(pos)].numpy(), atol=1e-12)
+
+
+ALL_CHECKS = [check_probe_rows_are_causal_softmax_rows, check_near_threshold_band, check_token_rows_equal_full_token_mask_attention,
               check_probe_positions_are_uniform_and_end_at_the_last_token,
               check_alpha_zero_is_dense_causal_attention, check_planted_vertical_and_slash_are_found,
               check_token_masked_attention_matches_brute_force, check_threshold_edges,
@@ -155,6 +172,10 @@ def test_aggregation_over_probes_is_the_max():
 
 def test_near_threshold_band():
     check_near_threshold_band()
+
+
+def test_probe_rows_are_causal_softmax_rows():
+    check_probe_rows_are_causal_softmax_rows()
 
 
 def test_token_rows_equal_full_token_mask_attention():
