@@ -19,6 +19,10 @@ CASES = {
     "tc_bf16_sparse": BASE.with_(seqlens=(1500,), hq=4, hkv=2, q_gain=40.0),
     "tc_bf16_varlen": BASE.with_(seqlens=(300, 0, 129, 640, 1, 128), hq=4, hkv=1, q_gain=20.0),
     "tc_bf16_gqa8": BASE.with_(seqlens=(777,), hq=8, hkv=1),
+    # odd GQA group (the last unit of each KV head holds one tile) and plain MHA (every unit
+    # holds one tile)
+    "tc_bf16_gqa3": BASE.with_(seqlens=(650, 129), hq=6, hkv=2, q_gain=30.0),
+    "tc_e4m3_mha": BASE.with_(seqlens=(400,), hq=2, hkv=2, dtype="e4m3", q_gain=20.0),
     "tc_e4m3": BASE.with_(seqlens=(900,), hq=2, hkv=1, dtype="e4m3", q_gain=20.0),
     # CUDA-core path
     "simt_f32_tiny": WORKLOADS["tiny_fp32_n2048"].with_(seqlens=(333,)),

@@ -128,6 +128,10 @@ CASES = {
     "e4m3": (BASE.with_(seqlens=(900,), hq=2, hkv=1, dtype="e4m3", q_gain=20.0), 32, 0.01, 0.01),
     "one_tile_group1": (BASE.with_(seqlens=(1100,), hq=2, hkv=2, q_gain=40.0), 64, 0.05, 0.02),
     "three_tiles": (BASE.with_(seqlens=(1300,), hq=4, hkv=1, q_gain=40.0), 96, 0.01, 0.01),
+    # odd group: 3 x 48 probe rows = one full tile and 16 rows; the attention's last unit of
+    # each KV head holds one tile
+    "gqa3_partial_tile": (BASE.with_(seqlens=(800, 333), hq=6, hkv=2, q_gain=40.0), 48, 0.01,
+                          0.01),
     "four_tiles_gqa8": (BASE.with_(seqlens=(1000,), hq=8, hkv=1, q_gain=40.0), 64, 0.01, 0.01),
     "alpha_zero_is_dense": (BASE.with_(seqlens=(700,), hq=2, hkv=1), 8, 0.0, 0.0),
     "alpha_above_one_is_empty": (BASE.with_(seqlens=(500, 300), hq=2, hkv=1, q_gain=40.0), 8,
