@@ -86,6 +86,8 @@ WORKLOADS: Dict[str, Workload] = {
                                      0.1, vertical_frac=0.002),
     "llama8b_e4m3_n131072": Workload("llama8b_e4m3_n131072", (131072,), 32, 8, 128, 128, "e4m3",
                                      0.1, vertical_frac=0.002),
+    # the e4m3 layer at 32K tokens (its Q + K + V, 200 MB, still exceed L2): kernel captures
+    "llama8b_e4m3_n32768": Workload("llama8b_e4m3_n32768", (32768,), 32, 8, 128, 128, "e4m3", 0.1),
     # packed varlen batch of eight sequences (continuous-batching shape)
     "varlen8_bf16_t264192": Workload("varlen8_bf16_t264192",
                                      (4096, 8192, 16384, 65536, 2048, 32768, 4096, 131072),
