@@ -436,6 +436,45 @@ class Prefill:
         res.update(self.selection())
         return res
 
+    def measure_graph(self, steps):
+        """The same search and attention replayed from two captured CUDA graphs (one launch
+        each from the host: what a server that replays its prefill graph sees), CUDA events
+        around each replay, L2 flushed before every step as in measure()."""
+        fpx, w, d = self.fpx, self.w, self.dev
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        g_search, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_search, stream=s):
+            fpx.block_scores(self.pf, d["q"], d["k"], self.ws, scores=self.scores)
+            fpx.select(self.pf, self.scores, w.alpha, self.ws, w.sink_blocks, w.window_blocks,
+                       row_ptr=self.row_ptr, col_idx=self.col_idx, nnz=self.nnz)
+        with torch.cuda.graph(g_attn, stream=s):
+            fpx.sparse_prefill(self.pf, d["q"], d["k"], d["v"], self.row_ptr, self.col_idx,
+                               self.ws, o=self.o, lse=self.lse)
+        flush = torch.empty(64 << 20, dtype=torch.float32, device=self.device)
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        for _ in range(3):
+            g_search.replay()
+            g_attn.replay()
+        torch.cuda.synchronize(self.device)
+        times = []
+        for _ in range(steps):
+            flush.fill_(0.0)
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record()
+            g_search.replay()
+            e1.record()
+            g_attn.replay()
+            e2.record()
+            times.append((e0, e1, e2))
+        torch.cuda.synchronize(self.device)
+        self.check_status("after the graph replays")
+        srch = statistics.mean(a.elapsed_time(b) for a, b, c in times)
+        attn = statistics.mean(b.elapsed_time(c) for a, b, c in times)
+        del g_search, g_attn, flush
+        return {"search_ms": round(srch, 4), "attn_ms": round(attn, 4),
+                "how": "search and attention each replayed from a captured CUDA graph"}
+
     def selection(self):
         w = self.w
         st = selection_stats(self.scores, self.row_ptr, self.col_idx, self.cu, w.hq, w.hkv,
@@ -484,6 +523,8 @@ def sub_records(fpx, args, device, sdpa_ms_128k):
             w = w0 if a is None else w0.with_(alpha=a)
             run = Prefill(fpx, w, data, device)
             r = run.measure(steps, 3)
+            if name == "llama8b_bf16_n8192":
+                r["graph"] = run.measure_graph(steps)
             del run
             torch.cuda.empty_cache()
             out["configs"].append({"workload": w.name, "alpha": w.alpha, **r})
