@@ -31,6 +31,10 @@
  * Ownership.  The caller owns every buffer.  No entry point allocates, frees or synchronises
  *   (except fpx_query_status, which synchronises the stream it is given).  All work is enqueued
  *   on the caller's stream; the library keeps no state between calls and is re-entrant.
+ *   Hence every entry point but fpx_query_status can be captured in a CUDA graph (stream
+ *   capture) and replayed; the kernels' programmatic dependent launches become graph edges.
+ *   A replay reads the buffers' contents at replay time, so new inputs copied into the
+ *   captured buffers give that input's result.
  * Workspaces.  Each entry point takes a device workspace of at least fpx_workspace_bytes()
  *   bytes (256-byte aligned).  Its first 256 bytes are a status block: kernels record the first
  *   device-side error there (bounded-wait timeout, malformed cu_seqlens or CSR, capacity); the
