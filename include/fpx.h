@@ -32,7 +32,9 @@
  *   (except fpx_query_status, which synchronises the stream it is given).  All work is enqueued
  *   on the caller's stream; the library keeps no state between calls and is re-entrant.
  *   Hence every entry point but fpx_query_status can be captured in a CUDA graph (stream
- *   capture) and replayed; the kernels' programmatic dependent launches become graph edges.
+ *   capture) and replayed once it has run eagerly on the device (a first call resolves the
+ *   driver's tensor-map encoder and, for fpx_select_noalloc, the scratch address); the
+ *   kernels' programmatic dependent launches become graph edges.
  *   A replay reads the buffers' contents at replay time, so new inputs copied into the
  *   captured buffers give that input's result.
  * Workspaces.  Each entry point takes a device workspace of at least fpx_workspace_bytes()
