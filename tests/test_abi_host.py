@@ -99,6 +99,23 @@ def test_invalid_problems_are_rejected_on_the_host(name):
     assert rc in (-1, -2)
 
 
+def test_csr_beyond_int32_is_rejected_and_just_below_is_accepted():
+    """row_ptr / col_idx are int32: a problem whose worst-case CSR (Hq x TRI entries, alpha = 0)
+    would not fit is refused on the host before any launch; one just inside fits."""
+    lib = fpx.load()
+    a, big = 0x100000, 1 << 40
+    p, keep = make([2_000_000], hq=32, hkv=8)  # 32 x 15625*15626/2 = 3.9e9 entries
+    ref = ctypes.byref(p)
+    assert lib.fpx_num_blocks(ref) == 0
+    assert lib.fpx_workspace_bytes(ref, -1) == 0
+    assert lib.fpx_block_scores(ref, a, a, a, a, big, None) == -2
+    p, keep = make([1_048_576], hq=32, hkv=8)  # 32 x 8192*8193/2 = 1.07e9 entries
+    ref = ctypes.byref(p)
+    assert lib.fpx_num_blocks(ref) == 8192
+    assert lib.fpx_max_nnz(ref) == 32 * 8192 * 8193 // 2 < 2**31 - 1
+    assert lib.fpx_workspace_bytes(ref, -1) > 0
+
+
 def test_host_argument_errors():
     lib = fpx.load()
     p, keep = make([300])
