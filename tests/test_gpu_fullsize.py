@@ -37,6 +37,9 @@ CASES = [
     ("llama8b_bf16_n131072", None, 415.0),
     ("llama8b_e4m3_n131072", None, 340.0),
     ("varlen8_bf16_t264192", None, 340.0),
+    # one 1 048 576-token sequence (8192 blocks per row: the index arithmetic of every stage well
+    # past the other layers'), two heads, in the sparse regime so that the oracle's CSR stays small
+    ("llama8b_bf16_n131072", None, 415.0, dict(seqlens=(1048576,), hq=2, hkv=1)),
 ]
 
 
@@ -61,10 +64,15 @@ def sample_blocks(w, cu, rng):
     return sorted(set(picks)), lay
 
 
-@pytest.mark.parametrize("name,alpha,q_gain", CASES,
-                         ids=[f"{n}-a{a}-g{g:g}" for n, a, g in CASES])
-def test_full_size_parity(name, alpha, q_gain):
-    w = WORKLOADS[name].with_(q_gain=q_gain)
+CASES = [c if len(c) == 4 else (*c, None) for c in CASES]
+
+
+@pytest.mark.parametrize("name,alpha,q_gain,over", CASES,
+                         ids=[f"{n}-a{a}-g{g:g}" + ("-" + "-".join(f"{k}{v[0] if isinstance(v, tuple) else v}"
+                                                                    for k, v in o.items()) if o else "")
+                              for n, a, g, o in CASES])
+def test_full_size_parity(name, alpha, q_gain, over):
+    w = WORKLOADS[name].with_(q_gain=q_gain, **(over or {}))
     if alpha is not None:
         w = w.with_(alpha=alpha)
     data = generate(w, workers=default_workers())
